@@ -1,0 +1,383 @@
+"""Benchmark of the Stem sparse-attention prefill path on B200.
+
+One step = one pass of the whole hot path over one layer's synthetic inputs
+(stem_score -> stem_select -> bsa_prefill, i.e. what stem_attention runs), inputs
+resident in HBM.  Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Default workload: one Qwen3-8B-shaped layer at 128K tokens in FP8-e4m3, keep 25%.
+With N > 1 (torchrun) every rank runs its own replica (the path has no exchange
+step); the device time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_attention_oam_b200 import stem as S          # noqa: E402
+from block_sparse_attention_oam_b200 import workloads as W     # noqa: E402
+
+METRIC = "Stem prefill ms/layer at 128K, 25% budget; effective TFLOP/s vs B200 peak"
+BF16_DATASHEET_TFLOPS = 2250.0
+FP8_OVER_BF16 = 2.0          # nominal dense FP8 / BF16 tensor throughput ratio
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS_PER_STEP = 6         # pool(Q), pool(K), pool(V), score, select, bsa
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK, "fallback"
+
+
+def selected_flops(prob: S.Problem, row_ptr: np.ndarray, block: int, head_dim: int, seqlens) -> float:
+    """Algorithmic FLOPs of the listed blocks: QK^T and PV over B x B tiles (2 x 2B^2 d),
+    the diagonal block counted as its causal half; ragged tails counted by valid tokens."""
+    flops = 0.0
+    row0 = 0
+    for S_ in seqlens:
+        N = math.ceil(S_ / block)
+        k = np.diff(row_ptr[row0: row0 + N + 1]).astype(np.float64)
+        rows = np.minimum(block, S_ - np.arange(N) * block).astype(np.float64)
+        # off-diagonal blocks: rows x block keys (the last block may be ragged only on the diagonal)
+        flops += float(np.sum((k - 1) * rows * block) * 4 * head_dim)
+        flops += float(np.sum(rows * (rows + 1) / 2) * 4 * head_dim)
+        row0 += N
+    return flops * prob.num_q_heads
+
+
+def dense_flops(seqlens, num_q_heads, head_dim):
+    return float(sum(s * (s + 1) / 2 for s in seqlens)) * 4 * head_dim * num_q_heads
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit()) if rows else None,
+                "reasons": sorted(reasons)}
+
+
+def cpu_baseline(inp: W.Inputs, rp: np.ndarray, ci: np.ndarray, budget_s: float = 15.0):
+    """Time the float64 oracle (as it stands) on a bounded sample of the workload on
+    the host cores and scale to ms per layer: pool + score + select for one q-head
+    (all rows), attention for a seeded subset of that head's q-blocks, extrapolated
+    by selected blocks to all heads."""
+    from oracle import stem_oracle as O
+    from threadpoolctl import threadpool_info
+    wl = inp.wl
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    h = 0
+    g = wl.num_q_heads // wl.num_kv_heads
+    t_sel = 0.0
+    t_att = 0.0
+    blocks_done = 0
+    blocks_total = int(ci.shape[1]) * wl.num_q_heads
+    rng = np.random.default_rng(0)
+    row0 = 0
+    cu = inp.cu_seqlens
+    sample_rows = 0
+    for b, S_ in enumerate(wl.seqlens):
+        t0, t1 = int(cu[b]), int(cu[b + 1])
+        N = math.ceil(S_ / wl.block)
+        q = inp.q[t0:t1, [h]].float().numpy().astype(np.float64) * inp.q_scale
+        k = inp.k[t0:t1, [h // g]].float().numpy().astype(np.float64) * inp.k_scale
+        v = inp.v[t0:t1, [h // g]].float().numpy().astype(np.float64) * inp.v_scale
+        c0 = time.perf_counter()
+        qbar, kbar, lbar = O.pool_mean(q, wl.block), O.pool_mean(k, wl.block), O.pool_log_norm(v, wl.block)
+        s = O.oam_scores(qbar, kbar, lbar, wl.softmax_scale, wl.beta)
+        kk = O.tpd_plan(N, wl.keep, wl.mu)[2]
+        lists = O.select_all(s, kk)
+        t_sel += (time.perf_counter() - c0) * wl.num_q_heads
+        order = rng.permutation(N)
+        c0 = time.perf_counter()
+        for i in order:
+            O.attend(q, k, v, lists, wl.block, wl.softmax_scale, rows=[(0, int(i))])
+            blocks_done += len(lists[0][i])
+            sample_rows += 1
+            if time.perf_counter() - c0 > budget_s / len(wl.seqlens):
+                break
+        t_att += time.perf_counter() - c0
+        row0 += N
+    ms = (t_sel + t_att * blocks_total / max(1, blocks_done)) * 1e3
+    return {"value": ms, "unit": "ms/layer", "cores": threads, "kind": "oracle",
+            "sample": f"float64 oracle on q-head 0: pool+score+select over all rows (x{wl.num_q_heads} heads), "
+                      f"attention on {sample_rows} seeded q-blocks ({blocks_done} of {blocks_total} selected "
+                      f"blocks), extrapolated by selected blocks"}
+
+
+def run_reference(args, wl):
+    """Reference arm: the oracle itself, timed as it stands on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    inp = W.make_inputs(wl)
+    from oracle import stem_oracle as O
+    # the oracle's own selection gives the CSR the sample needs
+    rows, cols = [], []
+    for S_ in wl.seqlens:
+        N = math.ceil(S_ / wl.block)
+        rows.append(O.tpd_plan(N, wl.keep, wl.mu)[2])
+    k = np.concatenate(rows)
+    rp = np.concatenate([[0], np.cumsum(k)]).astype(np.int32)
+    ci = np.zeros((wl.num_q_heads, int(rp[-1])), dtype=np.int32)
+    vals = []
+    for _ in range(args.warmup + args.steps):
+        vals.append(cpu_baseline(inp, rp, ci, budget_s=max(2.0, 20.0 / (args.warmup + args.steps))))
+    timed = vals[args.warmup:]
+    v = statistics.mean(x["value"] for x in timed)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "ms/layer", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": v, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "seq_len": list(wl.seqlens), "keep": wl.keep, "block": wl.block,
+                       "heads": [wl.num_q_heads, wl.num_kv_heads], "head_dim": wl.head_dim},
+            "cpu_baseline": {"value": v, "unit": "ms/layer", "cores": timed[-1]["cores"], "kind": "oracle",
+                             "sample": timed[-1]["sample"]},
+            "e2e": {"value": v, "unit": "ms/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=W.LONG_128K_FP8.name, choices=sorted(W.ALL))
+    ap.add_argument("--keep", type=float, default=None)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    wl = W.ALL[args.workload]
+    if args.keep is not None:
+        wl = wl.with_(keep=args.keep)
+    if args.impl == "reference":
+        run_reference(args, wl)
+        return
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the path has no CPU fallback)")
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    S.lib()
+
+    inp = W.make_inputs(wl.with_(seed=wl.seed + 1000 * rank))
+    prob = S.problem_for(wl, inp)
+    sz = prob.sizes()
+    q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
+    paged = None
+    if wl.paged:
+        paged = S.PagedKV(inp.k_cache.cuda(), inp.v_cache.cuda(), torch.from_numpy(inp.block_table).cuda())
+    ws = S.workspace(prob)
+    scores = torch.empty((wl.num_q_heads, sz["scores_per_head"]), dtype=torch.float32, device="cuda")
+    rp = torch.empty(sz["num_rows"] + 1, dtype=torch.int32, device="cuda")
+    ci = torch.empty((wl.num_q_heads, sz["nnz_per_head"]), dtype=torch.int32, device="cuda")
+    out = torch.empty((sz["total_tokens"], wl.num_q_heads, wl.head_dim), dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        S.stem_score(prob, q, k, v, paged, scores=scores, ws=ws)
+        if ev is not None:
+            ev[1].record(stream)
+        S.stem_select(prob, scores, rp, ci, ws=ws)
+        if ev is not None:
+            ev[2].record(stream)
+        S.bsa_prefill(prob, q, k, v, rp, ci, paged, out=out, ws=ws)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    S.query_status(ws)
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = Clocks(torch.cuda.current_device())
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if dist is not None:
+        dist.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    st_score = [e[0].elapsed_time(e[1]) for e in evs]
+    st_select = [e[1].elapsed_time(e[2]) for e in evs]
+    st_bsa = [e[2].elapsed_time(e[3]) for e in evs]
+    S.query_status(ws)
+    if dist is not None:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    rp_h = rp.cpu().numpy()
+    flops_sel = selected_flops(prob, rp_h, wl.block, wl.head_dim, wl.seqlens)
+    flops_dense = dense_flops(wl.seqlens, wl.num_q_heads, wl.head_dim)
+    bsa_ms = statistics.mean(st_bsa)
+    step_ms = total_ms / args.steps
+    peaks, peak_src = measured_peaks()
+    fp8 = wl.dtype == "fp8_e4m3"
+    peak = peaks["bf16_tflops_sustained"] * (FP8_OVER_BF16 if fp8 else 1.0)
+    achieved = flops_sel / (bsa_ms * 1e-3) / 1e12
+
+    result = {
+        "metric": METRIC, "value": step_ms / world, "unit": "ms/layer", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "seq_len": list(wl.seqlens), "keep": wl.keep, "mu": wl.mu,
+                   "beta": wl.beta, "block": wl.block, "heads": [wl.num_q_heads, wl.num_kv_heads],
+                   "head_dim": wl.head_dim, "paged": wl.paged, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (no flush)"},
+        "stages_ms": {"score": statistics.mean(st_score), "select": statistics.mean(st_select), "bsa": bsa_ms},
+        "score_select_frac": (statistics.mean(st_score) + statistics.mean(st_select)) / step_ms,
+        "selected_tflop": flops_sel / 1e12, "dense_tflop": flops_dense / 1e12,
+        "effective_tflops": {"bsa": achieved, "prefill": flops_sel / (step_ms * 1e-3) / 1e12,
+                             "bsa_frac_of_bf16_datasheet": achieved / BF16_DATASHEET_TFLOPS},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained" + (" x2 (fp8 nominal ratio)" if fp8 else ""),
+                     "kernel": "bsa_kernel"},
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clk,
+    }
+
+    if not args.no_dense:
+        dt = []
+        for i in range(3):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            S.bsa_dense_prefill(prob, q, k, v, paged, out=out, ws=ws)
+            b.record(stream)
+            torch.cuda.synchronize()
+            if i > 0:
+                dt.append(a.elapsed_time(b))
+        dense_ms = statistics.mean(dt)
+        result["dense"] = {"bsa_dense_ms": dense_ms, "speedup_prefill_vs_dense": dense_ms / step_ms,
+                           "dense_tflops": flops_dense / (dense_ms * 1e-3) / 1e12}
+        S.query_status(ws)
+
+    if not args.no_e2e:
+        # end to end through the public API with host buffers: H2D of Q/K/V (pinned),
+        # stem_attention, D2H of the output, every step.
+        hq, hk, hv = inp.q.pin_memory(), (inp.k_cache if wl.paged else inp.k).pin_memory(), \
+            (inp.v_cache if wl.paged else inp.v).pin_memory()
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        kd = paged.k_cache if wl.paged else k
+        vd = paged.v_cache if wl.paged else v
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            kd.copy_(hk, non_blocking=True)
+            vd.copy_(hv, non_blocking=True)
+            S.stem_attention(prob, q, k, v, paged, out=out, ws=ws)
+            hout.copy_(out, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, min(args.steps, 10))
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = a.elapsed_time(b) / n_e2e
+        if dist is not None:
+            t = torch.tensor([e2e_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        h2d = hq.numel() * hq.element_size() + hk.numel() * hk.element_size() + hv.numel() * hv.element_size()
+        result["e2e"] = {"value": e2e_ms / world, "unit": "ms/layer", "h2d_bytes_per_step": h2d,
+                         "d2h_bytes_per_step": hout.numel() * hout.element_size()}
+        S.query_status(ws)
+
+    if rank == 0 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(inp, rp_h, ci.cpu().numpy())
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+if __name__ == "__main__":
+    main()

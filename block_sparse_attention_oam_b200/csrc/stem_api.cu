@@ -1,0 +1,518 @@
+// libstem C-ABI: argument validation, the host TPD planner, workspace carve-up
+// and the entry points declared in include/stem.h.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <cmath>
+#include <map>
+#include <mutex>
+#include <tuple>
+#include <vector>
+
+#include "stem_internal.cuh"
+
+namespace stem {
+namespace {
+
+thread_local char g_err[512] = "";
+
+stem_status_t fail(stem_status_t s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+stem_status_t fail(stem_status_t s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+stem_status_t cuda_fail(cudaError_t e, const char* what) {
+  return fail(STEM_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// ------------------------------------------------------------- TPD planner
+// Tencent Cloud article "从Stem稀疏注意力看 大模型推理的架构取舍", section
+// "TPD：优先级排序": budget decays linearly, end = mu * start, total redistributed.
+// k_i(r) = min(i+1, max(m_i, floor(r * w_i))), w_i = (1 - (1-mu) i/(N-1)) (i+1),
+// m_i = min(2, i+1).  The plan is the midpoint of the first interval of r on which
+// the total reaches T; it is located by bisection on r, then pinned to the exact
+// jump values n / w_i that bound that interval.
+double tpd_weight(int N, double mu, int i) {
+  if (N == 1) return 1.0;
+  volatile double t = ((1.0 - mu) * static_cast<double>(i)) / static_cast<double>(N - 1);
+  return (1.0 - t) * static_cast<double>(i + 1);
+}
+
+struct Planner {
+  int N;
+  double mu;
+  std::vector<double> w;
+  Planner(int n, double m) : N(n), mu(m), w(n) {
+    for (int i = 0; i < n; ++i) w[i] = tpd_weight(n, m, i);
+  }
+  int64_t total(double r) const {
+    int64_t s = 0;
+    for (int i = 0; i < N; ++i) {
+      double f = floor(r * w[i]);
+      int64_t m = std::min(2, i + 1);
+      int64_t k = f < static_cast<double>(m) ? m : (f > static_cast<double>(i + 1) ? i + 1 : static_cast<int64_t>(f));
+      s += k;
+    }
+    return s;
+  }
+  // smallest jump value strictly greater than x (+inf if none)
+  double next_jump(double x) const {
+    double best = INFINITY;
+    for (int i = 0; i < N; ++i) {
+      const int lo_n = std::min(2, i + 1) + 1;
+      if (lo_n > i + 1) continue;
+      double f = floor(x * w[i]);
+      int64_t n = std::max<int64_t>(lo_n, static_cast<int64_t>(f < 0 ? 0 : f));
+      while (n > lo_n && static_cast<double>(n - 1) / w[i] > x) --n;
+      while (n <= i + 1 && static_cast<double>(n) / w[i] <= x) ++n;
+      if (n <= i + 1) best = std::min(best, static_cast<double>(n) / w[i]);
+    }
+    return best;
+  }
+  double last_jump() const {
+    double best = -INFINITY;
+    for (int i = 0; i < N; ++i)
+      if (std::min(2, i + 1) + 1 <= i + 1) best = std::max(best, static_cast<double>(i + 1) / w[i]);
+    return best;
+  }
+};
+
+int64_t tpd_target(int N, double keep) {
+  const int64_t C = static_cast<int64_t>(N) * (N + 1) / 2;
+  int64_t T = static_cast<int64_t>(floor(keep * static_cast<double>(C) + 0.5));
+  T = std::min(T, C);
+  T = std::max(T, static_cast<int64_t>(2) * N - 1);
+  return T;
+}
+
+void plan_uncached(int N, double keep, double mu, double* r_out, int64_t* total_out) {
+  Planner P(N, mu);
+  const int64_t T = tpd_target(N, keep);
+  const double first = P.next_jump(0.0);
+  if (!std::isfinite(first)) {  // no jumps at all (N <= 2)
+    *r_out = 1.0;
+    *total_out = P.total(1.0);
+    return;
+  }
+  if (P.total(first / 2.0) >= T) {
+    *r_out = first / 2.0;
+    *total_out = P.total(*r_out);
+    return;
+  }
+  double lo = 0.0, hi = 2.0 * P.last_jump();
+  for (int it = 0; it < 200; ++it) {
+    const double mid = 0.5 * (lo + hi);
+    if (mid <= lo || mid >= hi) break;
+    if (P.total(mid) >= T) hi = mid; else lo = mid;
+  }
+  // Walk the jump values from just below lo: the first interval whose midpoint
+  // total reaches T is the plan (midpoints sit far from any rounding-sensitive jump).
+  double J = P.next_jump(lo * (1.0 - 1e-12));
+  for (;;) {
+    const double J2 = P.next_jump(J);
+    const double mid = std::isfinite(J2) ? 0.5 * (J + J2) : 2.0 * J;
+    if (!std::isfinite(J2) || P.total(mid) >= T) {
+      *r_out = mid;
+      break;
+    }
+    J = J2;
+  }
+  *total_out = P.total(*r_out);
+}
+
+std::mutex g_plan_mu;
+std::map<std::tuple<int, double, double>, std::pair<double, int64_t>> g_plan_cache;
+
+void plan(int N, double keep, double mu, double* r, int64_t* total) {
+  const auto key = std::make_tuple(N, keep, mu);
+  {
+    std::lock_guard<std::mutex> g(g_plan_mu);
+    auto it = g_plan_cache.find(key);
+    if (it != g_plan_cache.end()) {
+      *r = it->second.first;
+      *total = it->second.second;
+      return;
+    }
+  }
+  plan_uncached(N, keep, mu, r, total);
+  std::lock_guard<std::mutex> g(g_plan_mu);
+  if (g_plan_cache.size() > 4096) g_plan_cache.clear();
+  g_plan_cache[key] = std::make_pair(*r, *total);
+}
+
+// ------------------------------------------------------------- validation
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+stem_status_t check_problem(const stem_problem_t* pr) {
+  if (pr == nullptr) return fail(STEM_ERR_INVALID, "problem is NULL");
+  if (pr->num_seqs < 1 || pr->num_seqs > STEM_MAX_SEQS)
+    return fail(STEM_ERR_INVALID, "num_seqs %d outside [1, %d]", pr->num_seqs, STEM_MAX_SEQS);
+  if (pr->cu_seqlens == nullptr) return fail(STEM_ERR_INVALID, "cu_seqlens is NULL");
+  if (pr->cu_seqlens[0] != 0) return fail(STEM_ERR_INVALID, "cu_seqlens[0] must be 0");
+  for (int b = 0; b < pr->num_seqs; ++b)
+    if (pr->cu_seqlens[b + 1] <= pr->cu_seqlens[b])
+      return fail(STEM_ERR_INVALID, "sequence %d has length %d", b, pr->cu_seqlens[b + 1] - pr->cu_seqlens[b]);
+  if (pr->num_q_heads < 1 || pr->num_kv_heads < 1 || pr->num_q_heads % pr->num_kv_heads != 0)
+    return fail(STEM_ERR_INVALID, "num_q_heads %d must be a positive multiple of num_kv_heads %d", pr->num_q_heads,
+                pr->num_kv_heads);
+  if (pr->num_q_heads > 256) return fail(STEM_ERR_UNSUPPORTED, "num_q_heads %d > 256", pr->num_q_heads);
+  if (pr->head_dim != 64 && pr->head_dim != 128)
+    return fail(STEM_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", pr->head_dim);
+  if (pr->block_size != 64 && pr->block_size != 128)
+    return fail(STEM_ERR_UNSUPPORTED, "block_size %d (supported: 64, 128)", pr->block_size);
+  if (pr->dtype != STEM_DT_BF16 && pr->dtype != STEM_DT_FP8_E4M3)
+    return fail(STEM_ERR_INVALID, "unknown dtype %d", static_cast<int>(pr->dtype));
+  if (pr->dtype == STEM_DT_FP8_E4M3) {
+    if (pr->head_dim != 128 || pr->block_size != 128)
+      return fail(STEM_ERR_UNSUPPORTED, "FP8 needs head_dim 128 and block_size 128");
+    if (!(pr->q_scale > 0.f) || !(pr->k_scale > 0.f) || !(pr->v_scale > 0.f) || !std::isfinite(pr->q_scale) ||
+        !std::isfinite(pr->k_scale) || !std::isfinite(pr->v_scale))
+      return fail(STEM_ERR_INVALID, "FP8 scales must be finite and positive");
+  }
+  if (!(pr->keep > 0.0 && pr->keep <= 1.0)) return fail(STEM_ERR_INVALID, "keep %g outside (0, 1]", pr->keep);
+  if (!(pr->mu > 0.0 && pr->mu <= 1.0)) return fail(STEM_ERR_INVALID, "mu %g outside (0, 1]", pr->mu);
+  if (!std::isfinite(pr->beta)) return fail(STEM_ERR_INVALID, "beta is not finite");
+  if (!std::isfinite(pr->softmax_scale)) return fail(STEM_ERR_INVALID, "softmax_scale is not finite");
+  long long T = pr->cu_seqlens[pr->num_seqs];
+  if (T > (1ll << 30)) return fail(STEM_ERR_UNSUPPORTED, "total tokens %lld too large", T);
+  for (int b = 0; b < pr->num_seqs; ++b) {
+    const int len = pr->cu_seqlens[b + 1] - pr->cu_seqlens[b];
+    const int nb = (len + pr->block_size - 1) / pr->block_size;
+    if (nb > STEM_MAX_BLOCKS)
+      return fail(STEM_ERR_UNSUPPORTED, "sequence %d has %d blocks (max %d)", b, nb, STEM_MAX_BLOCKS);
+  }
+  return STEM_OK;
+}
+
+stem_status_t check_paged(const stem_problem_t* pr, const stem_paged_kv_t* pg) {
+  if (pg == nullptr) return STEM_OK;
+  if (pg->k_cache == nullptr || pg->v_cache == nullptr || pg->block_table == nullptr)
+    return fail(STEM_ERR_INVALID, "paged cache pointers must not be NULL");
+  if (!aligned16(pg->k_cache) || !aligned16(pg->v_cache))
+    return fail(STEM_ERR_INVALID, "paged caches must be 16-byte aligned");
+  if (pg->page_size != STEM_PAGE_SIZE)
+    return fail(STEM_ERR_UNSUPPORTED, "page_size %d (supported: %d)", pg->page_size, STEM_PAGE_SIZE);
+  if (pg->num_slots < 1) return fail(STEM_ERR_INVALID, "num_slots %d", pg->num_slots);
+  for (int b = 0; b < pr->num_seqs; ++b) {
+    const int len = pr->cu_seqlens[b + 1] - pr->cu_seqlens[b];
+    if ((len + STEM_PAGE_SIZE - 1) / STEM_PAGE_SIZE > pg->max_pages_per_seq)
+      return fail(STEM_ERR_INVALID, "sequence %d needs more than max_pages_per_seq=%d pages", b,
+                  pg->max_pages_per_seq);
+  }
+  return STEM_OK;
+}
+
+void build_batch(const stem_problem_t* pr, Batch* bt) {
+  memset(bt, 0, sizeof(*bt));
+  bt->num_seqs = pr->num_seqs;
+  bt->block = pr->block_size;
+  bt->mu = pr->mu;
+  bt->total_tokens = pr->cu_seqlens[pr->num_seqs];
+  int rows = 0;
+  long long sc = 0, nz = 0;
+  for (int b = 0; b < pr->num_seqs; ++b) {
+    SeqInfo& s = bt->seq[b];
+    s.tok0 = pr->cu_seqlens[b];
+    s.len = pr->cu_seqlens[b + 1] - pr->cu_seqlens[b];
+    s.nblk = (s.len + pr->block_size - 1) / pr->block_size;
+    s.row0 = rows;
+    s.score0 = sc;
+    s.nnz0 = nz;
+    int64_t tot = 0;
+    plan(s.nblk, pr->keep, pr->mu, &s.r_start, &tot);
+    s.nnz = tot;
+    rows += s.nblk;
+    sc += static_cast<long long>(s.nblk) * (s.nblk + 1) / 2;
+    nz += tot;
+  }
+  bt->total_rows = rows;
+  bt->scores_per_head = sc;
+  bt->nnz_per_head = nz;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+WsLayout layout(const stem_problem_t* pr, const Batch& bt) {
+  WsLayout L;
+  size_t o = 0;
+  L.status = o;
+  o += 256;
+  const size_t R = static_cast<size_t>(bt.total_rows), d = static_cast<size_t>(pr->head_dim);
+  L.qbar = o;
+  o = align256(o + static_cast<size_t>(pr->num_q_heads) * R * d * 4);
+  L.kbar = o;
+  o = align256(o + static_cast<size_t>(pr->num_kv_heads) * R * d * 4);
+  L.lbar = o;
+  o = align256(o + static_cast<size_t>(pr->num_kv_heads) * R * 4);
+  L.scores = o;
+  o = align256(o + static_cast<size_t>(pr->num_q_heads) * static_cast<size_t>(bt.scores_per_head) * 4);
+  L.row_ptr = o;
+  o = align256(o + (R + 1) * 4);
+  L.col_idx = o;
+  o = align256(o + static_cast<size_t>(pr->num_q_heads) * static_cast<size_t>(bt.nnz_per_head) * 4);
+  L.total = o;
+  return L;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<unsigned char*>(ws) + off);
+}
+
+float sigma_of(const stem_problem_t* pr) {
+  return pr->softmax_scale > 0.f ? pr->softmax_scale : 1.0f / sqrtf(static_cast<float>(pr->head_dim));
+}
+
+stem_status_t check_ws(const stem_problem_t* pr, const Batch& bt, void* ws, size_t ws_bytes, WsLayout* L) {
+  *L = layout(pr, bt);
+  if (ws == nullptr) return fail(STEM_ERR_WORKSPACE, "workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(STEM_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (ws_bytes < L->total)
+    return fail(STEM_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, L->total);
+  return STEM_OK;
+}
+
+stem_status_t do_score(const stem_problem_t* pr, const Batch& bt, const WsLayout& L, const void* q, const void* k,
+                       const void* v, const stem_paged_kv_t* pg, float* scores, void* ws, cudaStream_t st) {
+  const bool fp8 = pr->dtype == STEM_DT_FP8_E4M3;
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  PoolArgs a{};
+  a.x = q;
+  a.H = pr->num_q_heads;
+  a.scale = fp8 ? pr->q_scale : 1.0f;
+  a.mean_out = at<float>(ws, L.qbar);
+  a.lognorm_out = nullptr;
+  cudaError_t e = launch_pool(bt, a, pr->head_dim, fp8, false, status, st);
+  if (e != cudaSuccess) return cuda_fail(e, "pool(Q)");
+  PoolArgs kk{};
+  kk.x = pg ? pg->k_cache : k;
+  kk.block_table = pg ? pg->block_table : nullptr;
+  kk.max_pages = pg ? pg->max_pages_per_seq : 0;
+  kk.H = pr->num_kv_heads;
+  kk.scale = fp8 ? pr->k_scale : 1.0f;
+  kk.mean_out = at<float>(ws, L.kbar);
+  kk.lognorm_out = nullptr;
+  e = launch_pool(bt, kk, pr->head_dim, fp8, pg != nullptr, status, st);
+  if (e != cudaSuccess) return cuda_fail(e, "pool(K)");
+  PoolArgs vv = kk;
+  vv.x = pg ? pg->v_cache : v;
+  vv.scale = fp8 ? pr->v_scale : 1.0f;
+  vv.mean_out = nullptr;
+  vv.lognorm_out = at<float>(ws, L.lbar);
+  e = launch_pool(bt, vv, pr->head_dim, fp8, pg != nullptr, status, st);
+  if (e != cudaSuccess) return cuda_fail(e, "pool(V)");
+  e = launch_score(bt, at<float>(ws, L.qbar), at<float>(ws, L.kbar), at<float>(ws, L.lbar), pr->num_q_heads,
+                   pr->num_kv_heads, pr->head_dim, sigma_of(pr), pr->beta, scores, st);
+  if (e != cudaSuccess) return cuda_fail(e, "score");
+  return STEM_OK;
+}
+
+stem_status_t do_bsa(const stem_problem_t* pr, const Batch& bt, const WsLayout& L, const void* q, const void* k,
+                     const void* v, const stem_paged_kv_t* pg, const int32_t* row_ptr, const int32_t* col_idx,
+                     void* out, float* lse, void* ws, bool dense, cudaStream_t st) {
+  BsaArgs a{};
+  a.q = q;
+  a.k = pg ? pg->k_cache : k;
+  a.v = pg ? pg->v_cache : v;
+  a.block_table = pg ? pg->block_table : nullptr;
+  a.max_pages = pg ? pg->max_pages_per_seq : 0;
+  a.kv_rows = pg ? static_cast<long long>(pg->num_slots) * STEM_PAGE_SIZE : bt.total_tokens;
+  a.row_ptr = row_ptr;
+  a.col_idx = col_idx;
+  a.out = out;
+  a.lse = lse;
+  a.Hq = pr->num_q_heads;
+  a.Hkv = pr->num_kv_heads;
+  a.head_dim = pr->head_dim;
+  a.sigma = sigma_of(pr);
+  a.q_scale = pr->q_scale;
+  a.k_scale = pr->k_scale;
+  a.v_scale = pr->v_scale;
+  cudaError_t e = launch_bsa(bt, a, pr->dtype == STEM_DT_FP8_E4M3, pg != nullptr, dense, at<uint32_t>(ws, L.status), st);
+  if (e != cudaSuccess) return cuda_fail(e, dense ? "bsa_dense" : "bsa");
+  return STEM_OK;
+}
+
+stem_status_t check_qkv(const void* q, const void* k, const void* v, const stem_paged_kv_t* pg) {
+  if (q == nullptr || !aligned16(q)) return fail(STEM_ERR_INVALID, "q must be a non-NULL 16-byte aligned pointer");
+  if (pg == nullptr) {
+    if (k == nullptr || v == nullptr || !aligned16(k) || !aligned16(v))
+      return fail(STEM_ERR_INVALID, "k and v must be non-NULL 16-byte aligned pointers");
+  }
+  return STEM_OK;
+}
+
+}  // namespace
+}  // namespace stem
+
+using namespace stem;
+
+extern "C" {
+
+stem_status_t stem_query_sizes(const stem_problem_t* prob, stem_sizes_t* out) {
+  stem_status_t s = check_problem(prob);
+  if (s != STEM_OK) return s;
+  if (out == nullptr) return fail(STEM_ERR_INVALID, "out is NULL");
+  Batch bt;
+  build_batch(prob, &bt);
+  WsLayout L = layout(prob, bt);
+  out->num_rows = bt.total_rows;
+  out->scores_per_head = bt.scores_per_head;
+  out->nnz_per_head = bt.nnz_per_head;
+  out->total_tokens = bt.total_tokens;
+  out->workspace_bytes = L.total;
+  return STEM_OK;
+}
+
+size_t stem_workspace_size(const stem_problem_t* prob) {
+  stem_sizes_t s;
+  return stem_query_sizes(prob, &s) == STEM_OK ? s.workspace_bytes : 0;
+}
+
+stem_status_t stem_tpd_plan(int n_blocks, double keep, double mu, double* r_start, int64_t* total) {
+  if (n_blocks < 1) return fail(STEM_ERR_INVALID, "n_blocks %d < 1", n_blocks);
+  if (!(keep > 0.0 && keep <= 1.0)) return fail(STEM_ERR_INVALID, "keep %g outside (0, 1]", keep);
+  if (!(mu > 0.0 && mu <= 1.0)) return fail(STEM_ERR_INVALID, "mu %g outside (0, 1]", mu);
+  if (r_start == nullptr || total == nullptr) return fail(STEM_ERR_INVALID, "output pointer is NULL");
+  plan(n_blocks, keep, mu, r_start, total);
+  return STEM_OK;
+}
+
+stem_status_t stem_score(const stem_problem_t* prob, const void* q, const void* k, const void* v,
+                         const stem_paged_kv_t* paged, float* scores, void* ws, size_t ws_bytes, void* stream) {
+  stem_status_t s = check_problem(prob);
+  if (s == STEM_OK) s = check_paged(prob, paged);
+  if (s == STEM_OK) s = check_qkv(q, k, v, paged);
+  if (s != STEM_OK) return s;
+  if (scores == nullptr) return fail(STEM_ERR_INVALID, "scores is NULL");
+  Batch bt;
+  build_batch(prob, &bt);
+  WsLayout L;
+  if ((s = check_ws(prob, bt, ws, ws_bytes, &L)) != STEM_OK) return s;
+  return do_score(prob, bt, L, q, k, v, paged, scores, ws, static_cast<cudaStream_t>(stream));
+}
+
+stem_status_t stem_select(const stem_problem_t* prob, const float* scores, int32_t* row_ptr, int32_t* col_idx,
+                          void* ws, size_t ws_bytes, void* stream) {
+  stem_status_t s = check_problem(prob);
+  if (s != STEM_OK) return s;
+  if (scores == nullptr || row_ptr == nullptr || col_idx == nullptr)
+    return fail(STEM_ERR_INVALID, "scores, row_ptr and col_idx must not be NULL");
+  Batch bt;
+  build_batch(prob, &bt);
+  WsLayout L;
+  if ((s = check_ws(prob, bt, ws, ws_bytes, &L)) != STEM_OK) return s;
+  cudaError_t e = launch_select(bt, scores, prob->num_q_heads, row_ptr, col_idx, at<uint32_t>(ws, L.status),
+                                static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "select");
+  return STEM_OK;
+}
+
+stem_status_t bsa_prefill(const stem_problem_t* prob, const void* q, const void* k, const void* v,
+                          const stem_paged_kv_t* paged, const int32_t* row_ptr, const int32_t* col_idx, void* out,
+                          float* lse, void* ws, size_t ws_bytes, void* stream) {
+  stem_status_t s = check_problem(prob);
+  if (s == STEM_OK) s = check_paged(prob, paged);
+  if (s == STEM_OK) s = check_qkv(q, k, v, paged);
+  if (s != STEM_OK) return s;
+  if (row_ptr == nullptr || col_idx == nullptr) return fail(STEM_ERR_INVALID, "row_ptr and col_idx must not be NULL");
+  if (out == nullptr || !aligned16(out)) return fail(STEM_ERR_INVALID, "out must be a non-NULL 16-byte aligned pointer");
+  Batch bt;
+  build_batch(prob, &bt);
+  WsLayout L;
+  if ((s = check_ws(prob, bt, ws, ws_bytes, &L)) != STEM_OK) return s;
+  return do_bsa(prob, bt, L, q, k, v, paged, row_ptr, col_idx, out, lse, ws, false, static_cast<cudaStream_t>(stream));
+}
+
+stem_status_t bsa_dense_prefill(const stem_problem_t* prob, const void* q, const void* k, const void* v,
+                                const stem_paged_kv_t* paged, void* out, float* lse, void* ws, size_t ws_bytes,
+                                void* stream) {
+  stem_status_t s = check_problem(prob);
+  if (s == STEM_OK) s = check_paged(prob, paged);
+  if (s == STEM_OK) s = check_qkv(q, k, v, paged);
+  if (s != STEM_OK) return s;
+  if (out == nullptr || !aligned16(out)) return fail(STEM_ERR_INVALID, "out must be a non-NULL 16-byte aligned pointer");
+  Batch bt;
+  build_batch(prob, &bt);
+  WsLayout L;
+  if ((s = check_ws(prob, bt, ws, ws_bytes, &L)) != STEM_OK) return s;
+  return do_bsa(prob, bt, L, q, k, v, paged, nullptr, nullptr, out, lse, ws, true, static_cast<cudaStream_t>(stream));
+}
+
+stem_status_t stem_attention(const stem_problem_t* prob, const void* q, const void* k, const void* v,
+                             const stem_paged_kv_t* paged, void* out, float* lse, int32_t* row_ptr_out,
+                             int32_t* col_idx_out, void* ws, size_t ws_bytes, void* stream) {
+  stem_status_t s = check_problem(prob);
+  if (s == STEM_OK) s = check_paged(prob, paged);
+  if (s == STEM_OK) s = check_qkv(q, k, v, paged);
+  if (s != STEM_OK) return s;
+  if (out == nullptr || !aligned16(out)) return fail(STEM_ERR_INVALID, "out must be a non-NULL 16-byte aligned pointer");
+  Batch bt;
+  build_batch(prob, &bt);
+  WsLayout L;
+  if ((s = check_ws(prob, bt, ws, ws_bytes, &L)) != STEM_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* scores = at<float>(ws, L.scores);
+  int32_t* rp = at<int32_t>(ws, L.row_ptr);
+  int32_t* ci = at<int32_t>(ws, L.col_idx);
+  if ((s = do_score(prob, bt, L, q, k, v, paged, scores, ws, st)) != STEM_OK) return s;
+  cudaError_t e = launch_select(bt, scores, prob->num_q_heads, rp, ci, at<uint32_t>(ws, L.status), st);
+  if (e != cudaSuccess) return cuda_fail(e, "select");
+  if ((s = do_bsa(prob, bt, L, q, k, v, paged, rp, ci, out, lse, ws, false, st)) != STEM_OK) return s;
+  if (row_ptr_out != nullptr) {
+    e = cudaMemcpyAsync(row_ptr_out, rp, (static_cast<size_t>(bt.total_rows) + 1) * 4, cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "copy row_ptr");
+  }
+  if (col_idx_out != nullptr) {
+    e = cudaMemcpyAsync(col_idx_out, ci, static_cast<size_t>(prob->num_q_heads) * bt.nnz_per_head * 4,
+                        cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "copy col_idx");
+  }
+  return STEM_OK;
+}
+
+stem_status_t stem_query_status(void* ws, void* stream) {
+  if (ws == nullptr) return fail(STEM_ERR_WORKSPACE, "workspace is NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  uint32_t word = 0;
+  e = cudaMemcpy(&word, ws, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read status");
+  e = cudaMemset(ws, 0, sizeof(word));
+  if (e != cudaSuccess) return cuda_fail(e, "clear status");
+  if (word & kStatusTimeout) return fail(STEM_ERR_TIMEOUT, "a device pipeline wait timed out");
+  if (word & kStatusBounds) return fail(STEM_ERR_BOUNDS, "a block index outside its sequence was seen");
+  return STEM_OK;
+}
+
+stem_status_t stem_reset_status(void* ws, void* stream) {
+  if (ws == nullptr) return fail(STEM_ERR_WORKSPACE, "workspace is NULL");
+  cudaError_t e = cudaMemsetAsync(ws, 0, 256, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "reset status");
+  return STEM_OK;
+}
+
+const char* stem_status_string(stem_status_t s) {
+  switch (s) {
+    case STEM_OK: return "ok";
+    case STEM_ERR_INVALID: return "invalid argument";
+    case STEM_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case STEM_ERR_WORKSPACE: return "workspace missing or too small";
+    case STEM_ERR_CUDA: return "CUDA error";
+    case STEM_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case STEM_ERR_BOUNDS: return "block index out of range";
+  }
+  return "unknown status";
+}
+
+const char* stem_last_error(void) { return g_err; }
+
+}  // extern "C"

@@ -1,0 +1,249 @@
+// OAM scoring on sm_100a: the per-block pooling kernel and the block-score GEMM.
+//
+// Tencent Cloud article "从Stem稀疏注意力看 大模型推理的架构取舍":
+//  * section "OAM：价值评估": score = routing relevance (QK^T) + beta * log||V_j||_2,
+//    beta = 0.2, purely additive;
+//  * section "HPC-Stem：评估选块，快几十倍": because the score is additive, compact
+//    block-level representations of Q and K are computed first and one standard
+//    GEMM yields every block score, with no softmax, no gather and no large
+//    intermediate tensor.
+// The block summary is the mean over the block's tokens; the magnitude term is the
+// block mean of the per-token log L2 norm of V (zero norms clamped to FLT_MIN).
+#include <cuda_fp16.h>
+#include <float.h>
+
+#include "stem_internal.cuh"
+
+namespace stem {
+namespace {
+
+constexpr int kPoolThreads = 128;
+
+__device__ __forceinline__ void decode16(const uint4& u, float* f, bool fp8, float scale) {
+  if (!fp8) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      f[2 * q] = __uint_as_float(w[q] << 16);
+      f[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
+    }
+  } else {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+      for (int hlf = 0; hlf < 2; ++hlf) {
+        uint16_t pair = static_cast<uint16_t>(w[q] >> (16 * hlf));
+        uint32_t h2;
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
+        __half2 hv = *reinterpret_cast<__half2*>(&h2);
+        float2 fv = __half22float2(hv);
+        f[4 * q + 2 * hlf] = fv.x * scale;
+        f[4 * q + 2 * hlf + 1] = fv.y * scale;
+      }
+    }
+  }
+}
+
+// One CTA per (global block row, group of 128 x VEC elements of the [H*d] token row).
+// Each thread owns VEC consecutive elements (16 bytes) of one head and walks the
+// block's tokens, so every warp reads 512 contiguous bytes per token.
+template <int D, bool FP8, bool PAGED>
+__global__ void __launch_bounds__(kPoolThreads) pool_kernel(const Batch bt, PoolArgs a) {
+  constexpr int VEC = FP8 ? 16 : 8;
+  constexpr int LPH = D / VEC;  // lanes per head
+  const int row = blockIdx.x;
+  const int b = seq_of_row(bt, row);
+  const SeqInfo& s = bt.seq[b];
+  const int i = row - s.row0;
+  const int B = bt.block;
+  const int t_beg = i * B;
+  const int t_end = min(s.len, t_beg + B);
+  const int n = t_end - t_beg;
+  const int HD = a.H * D;
+  const int e0 = (blockIdx.y * kPoolThreads + threadIdx.x) * VEC;
+  const bool valid = e0 < HD;
+  const int h = valid ? e0 / D : 0;
+  const int d0 = e0 % D;
+  const unsigned char* base = static_cast<const unsigned char*>(a.x);
+  constexpr int ES = FP8 ? 1 : 2;
+
+  float acc[VEC];
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+  float lacc = 0.f;
+
+  auto tok_ptr = [&](int t) -> const uint4* {
+    long long rowi;
+    if (PAGED) {
+      int slot = a.block_table[static_cast<long long>(b) * a.max_pages + t / STEM_PAGE_SIZE];
+      rowi = static_cast<long long>(slot) * STEM_PAGE_SIZE + (t % STEM_PAGE_SIZE);
+    } else {
+      rowi = static_cast<long long>(s.tok0) + t;
+    }
+    return reinterpret_cast<const uint4*>(base + (rowi * HD + e0) * ES);
+  };
+
+  constexpr int U = 4;
+  for (int t = t_beg; t < t_end; t += U) {
+    uint4 buf[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      buf[u] = make_uint4(0, 0, 0, 0);
+      if (valid && t + u < t_end) buf[u] = __ldg(tok_ptr(t + u));
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float f[VEC];
+      decode16(buf[u], f, FP8, a.scale);
+      float ss = 0.f;
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        acc[e] += f[e];
+        ss = fmaf(f[e], f[e], ss);
+      }
+      if (a.lognorm_out != nullptr) {
+#pragma unroll
+        for (int o = LPH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o, LPH);
+        if (t + u < t_end) lacc += logf(fmaxf(sqrtf(ss), FLT_MIN));
+      }
+    }
+  }
+  if (!valid) return;
+  const float inv = 1.0f / static_cast<float>(n);
+  float* dst = a.mean_out + (static_cast<long long>(h) * bt.total_rows + row) * D + d0;
+#pragma unroll
+  for (int e = 0; e < VEC; e += 4)
+    *reinterpret_cast<float4*>(dst + e) = make_float4(acc[e] * inv, acc[e + 1] * inv, acc[e + 2] * inv, acc[e + 3] * inv);
+  if (a.lognorm_out != nullptr && d0 == 0) a.lognorm_out[static_cast<long long>(h) * bt.total_rows + row] = lacc * inv;
+}
+
+template <int D, bool FP8>
+cudaError_t pool_dispatch_paged(const Batch& bt, const PoolArgs& a, bool paged, cudaStream_t st) {
+  constexpr int VEC = FP8 ? 16 : 8;
+  dim3 grid(bt.total_rows, (a.H * D + kPoolThreads * VEC - 1) / (kPoolThreads * VEC));
+  if (paged)
+    pool_kernel<D, FP8, true><<<grid, kPoolThreads, 0, st>>>(bt, a);
+  else
+    pool_kernel<D, FP8, false><<<grid, kPoolThreads, 0, st>>>(bt, a);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ scores
+// One CTA per (64 x 64 lower-triangular tile of one sequence, q-head).  fp32 SIMT:
+// the GEMM is N x N x d per head (about 4 GFLOP at 128K), far below the path's
+// cost, and fp32 keeps the scores within 1e-3 relative of the float64 definition.
+constexpr int kTile = 64;
+constexpr int kKc = 32;
+
+__global__ void __launch_bounds__(256) score_kernel(const Batch bt, const float* __restrict__ qbar,
+                                                    const float* __restrict__ kbar,
+                                                    const float* __restrict__ lbar, int Hq, int Hkv, int D,
+                                                    float sigma, float beta, float* __restrict__ scores) {
+  __shared__ float Qs[kKc][kTile + 1];
+  __shared__ float Ks[kKc][kTile + 1];
+  const int h = blockIdx.y;
+  const int kh = h / (Hq / Hkv);
+  // decode (sequence, tile row, tile col)
+  long long t = blockIdx.x;
+  int b = 0;
+  int nt = 0;
+  for (; b < bt.num_seqs; ++b) {
+    nt = (bt.seq[b].nblk + kTile - 1) / kTile;
+    long long cnt = static_cast<long long>(nt) * (nt + 1) / 2;
+    if (t < cnt) break;
+    t -= cnt;
+  }
+  if (b >= bt.num_seqs) return;
+  int ti = static_cast<int>((sqrt(8.0 * static_cast<double>(t) + 1.0) - 1.0) * 0.5);
+  while (static_cast<long long>(ti) * (ti + 1) / 2 > t) --ti;
+  while (static_cast<long long>(ti + 1) * (ti + 2) / 2 <= t) ++ti;
+  const int tj = static_cast<int>(t - static_cast<long long>(ti) * (ti + 1) / 2);
+  const SeqInfo& s = bt.seq[b];
+  const int N = s.nblk;
+  const int R = bt.total_rows;
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  const int i0 = ti * kTile, j0 = tj * kTile;
+
+  float acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
+
+  const float* qrow = qbar + (static_cast<long long>(h) * R + s.row0) * D;
+  const float* krow = kbar + (static_cast<long long>(kh) * R + s.row0) * D;
+  const int lr = threadIdx.x / 4;        // 0..63 tile row loaded by this thread
+  const int lc = (threadIdx.x % 4) * 8;  // 8 consecutive d of the chunk
+  for (int kc = 0; kc < D; kc += kKc) {
+    float4 qa = make_float4(0, 0, 0, 0), qb = qa, ka = qa, kb = qa;
+    if (i0 + lr < N) {
+      const float4* p = reinterpret_cast<const float4*>(qrow + static_cast<long long>(i0 + lr) * D + kc + lc);
+      qa = p[0];
+      qb = p[1];
+    }
+    if (j0 + lr < N) {
+      const float4* p = reinterpret_cast<const float4*>(krow + static_cast<long long>(j0 + lr) * D + kc + lc);
+      ka = p[0];
+      kb = p[1];
+    }
+    __syncthreads();
+    const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+    const float kv[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      Qs[lc + e][lr] = qv[e];
+      Ks[lc + e][lr] = kv[e];
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < kKc; ++kk) {
+      float av[4], bv[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) av[a] = Qs[kk][ty + 16 * a];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) bv[c] = Ks[kk][tx + 16 * c];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[a][c] = fmaf(av[a], bv[c], acc[a][c]);
+    }
+  }
+  float* out = scores + static_cast<long long>(h) * bt.scores_per_head + s.score0;
+  const float* lb = lbar + static_cast<long long>(kh) * R + s.row0;
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int i = i0 + ty + 16 * a;
+    if (i >= N) continue;
+    const long long roff = static_cast<long long>(i) * (i + 1) / 2;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int j = j0 + tx + 16 * c;
+      if (j <= i) out[roff + j] = fmaf(sigma, acc[a][c], beta * lb[j]);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_pool(const Batch& bt, const PoolArgs& a, int head_dim, bool fp8, bool paged, uint32_t*,
+                        cudaStream_t st) {
+  if (head_dim == 128) return fp8 ? pool_dispatch_paged<128, true>(bt, a, paged, st)
+                                  : pool_dispatch_paged<128, false>(bt, a, paged, st);
+  if (head_dim == 64 && !fp8) return pool_dispatch_paged<64, false>(bt, a, paged, st);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_score(const Batch& bt, const float* qbar, const float* kbar, const float* lbar, int Hq, int Hkv,
+                         int head_dim, float sigma, float beta, float* scores, cudaStream_t st) {
+  long long tiles = 0;
+  for (int b = 0; b < bt.num_seqs; ++b) {
+    long long nt = (bt.seq[b].nblk + kTile - 1) / kTile;
+    tiles += nt * (nt + 1) / 2;
+  }
+  dim3 grid(static_cast<unsigned>(tiles), Hq);
+  score_kernel<<<grid, 256, 0, st>>>(bt, qbar, kbar, lbar, Hq, Hkv, head_dim, sigma, beta, scores);
+  return cudaGetLastError();
+}
+
+}  // namespace stem

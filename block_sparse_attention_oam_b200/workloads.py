@@ -128,7 +128,8 @@ def _gen_sequence(wl: Workload, seq_index: int, S: int):
 
 def _quant_fp8(x_bf16: torch.Tensor):
     amax = float(x_bf16.float().abs().max())
-    scale = amax / FP8_E4M3_MAX if amax > 0 else 1.0
+    # a float32-representable scale, so host (float64) and device (float32) agree exactly
+    scale = float(np.float32(amax / FP8_E4M3_MAX)) if amax > 0 else 1.0
     codes = (x_bf16.float() / scale).to(torch.float8_e4m3fn)
     return codes, scale
 
