@@ -80,7 +80,7 @@ struct BsaParams {
   int Hq, Hkv;
   int total_tiles;
   float scale_log2;  // sigma * q_scale * k_scale * log2(e)
-  float out_scale;   // v_scale / p_scale
+  float out_scale;   // FP8: v_scale (l carries p_scale); BF16: 1
   float p_scale;     // FP8: P is multiplied by this before rounding to e4m3
   uint32_t* status;
   signed char order[STEM_MAX_SEQS];  // sequences by decreasing block count
@@ -415,8 +415,9 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
             for (int e = 0; e < 4; ++e) {
               const float p0 = ex2_approx(fmaf(__uint_as_float(sr[8 * u + 2 * e]), p.scale_log2, -m_use));
               const float p1 = ex2_approx(fmaf(__uint_as_float(sr[8 * u + 2 * e + 1]), p.scale_log2, -m_use));
-              sum += p0 + p1;
               w4[e] = pack_bf16x2(p0, p1);
+              // normalise with the rounded weights the P.V product uses
+              sum += __uint_as_float(w4[e] << 16) + __uint_as_float(w4[e] & 0xFFFF0000u);
             }
             const int chunk = u / 8, uu = u % 8;
             const uint32_t addr = pbuf + chunk * C::Q_CHUNK + r * 128 + ((uu ^ (r & 7)) << 4);
@@ -432,12 +433,15 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
             for (int e = 0; e < 4; ++e) {
               float pv[4];
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
+              for (int q = 0; q < 4; ++q)
                 pv[q] = ex2_approx(fmaf(__uint_as_float(sr[16 * u + 4 * e + q]), p.scale_log2, -m_use));
-                sum += pv[q];
-              }
-              w4[e] = pack_e4m3x2(pv[0] * p.p_scale, pv[1] * p.p_scale) |
-                      (pack_e4m3x2(pv[2] * p.p_scale, pv[3] * p.p_scale) << 16);
+              const uint32_t lo = pack_e4m3x2(pv[0] * p.p_scale, pv[1] * p.p_scale);
+              const uint32_t hi = pack_e4m3x2(pv[2] * p.p_scale, pv[3] * p.p_scale);
+              w4[e] = lo | (hi << 16);
+              // normalise with the rounded (scaled) weights the P.V product uses
+              const float2 a = e4m3x2_to_float2(static_cast<uint16_t>(lo));
+              const float2 b = e4m3x2_to_float2(static_cast<uint16_t>(hi));
+              sum += (a.x + a.y) + (b.x + b.y);
             }
             const uint32_t addr = pbuf + r * 128 + ((u ^ (r & 7)) << 4);
             asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w4[0]), "r"(w4[1]), "r"(w4[2]),
@@ -498,7 +502,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
         }
       }
       if (p.lse != nullptr && r < rows_valid)
-        p.lse[static_cast<long long>(tl.h) * p.bt.total_tokens + tok] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+        p.lse[static_cast<long long>(tl.h) * p.bt.total_tokens + tok] =
+            (m_run + __log2f(l_run / p.p_scale)) * 0.69314718055994531f;
       tc_fence_before();
     }
   }
@@ -590,7 +595,8 @@ cudaError_t launch_bsa(const Batch& bt, const BsaArgs& a, bool fp8, bool paged, 
   prm.scale_log2 = a.sigma * (fp8 ? a.q_scale * a.k_scale : 1.0f) * log2e;
   // FP8: P <= 2^8 after the lazy max update; 448 / 256 keeps it inside e4m3's range.
   prm.p_scale = fp8 ? 1.75f : 1.0f;
-  prm.out_scale = fp8 ? a.v_scale / prm.p_scale : 1.0f;
+  // l is accumulated from the scaled, rounded P, so the V scale is all that remains
+  prm.out_scale = fp8 ? a.v_scale : 1.0f;
   long long tiles = 0;
   for (int b = 0; b < bt.num_seqs; ++b) tiles += static_cast<long long>(bt.seq[b].nblk) * a.Hq;
   prm.total_tiles = static_cast<int>(tiles);

@@ -111,10 +111,13 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const Batch bt, Pool
   }
   if (!valid) return;
   const float inv = 1.0f / static_cast<float>(n);
-  float* dst = a.mean_out + (static_cast<long long>(h) * bt.total_rows + row) * D + d0;
+  if (a.mean_out != nullptr) {
+    float* dst = a.mean_out + (static_cast<long long>(h) * bt.total_rows + row) * D + d0;
 #pragma unroll
-  for (int e = 0; e < VEC; e += 4)
-    *reinterpret_cast<float4*>(dst + e) = make_float4(acc[e] * inv, acc[e + 1] * inv, acc[e + 2] * inv, acc[e + 3] * inv);
+    for (int e = 0; e < VEC; e += 4)
+      *reinterpret_cast<float4*>(dst + e) =
+          make_float4(acc[e] * inv, acc[e + 1] * inv, acc[e + 2] * inv, acc[e + 3] * inv);
+  }
   if (a.lognorm_out != nullptr && d0 == 0) a.lognorm_out[static_cast<long long>(h) * bt.total_rows + row] = lacc * inv;
 }
 

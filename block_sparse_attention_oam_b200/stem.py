@@ -168,7 +168,11 @@ class PagedKV:
 
 
 def _ptr(t: Optional[torch.Tensor]):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("libstem takes dense row-major tensors; got a non-contiguous one")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _stream(stream=None):

@@ -78,7 +78,7 @@ def test_select_bit_exact_on_oracle_scores(name, keep, mu):
     packed, lists = [], []
     for b, N in enumerate(_seq_blocks(wl)):
         s = T.oracle_scores(inp, b).astype(np.float32)            # the exact bytes both sides rank
-        packed.append(O.pack_causal(s))
+        packed.append(np.ascontiguousarray(O.pack_causal(s)))
         k = O.tpd_plan(N, keep, mu)[2]
         lists.append(O.select_all(s.astype(np.float64), k))
     scores = torch.from_numpy(np.concatenate(packed, axis=1)).cuda()
@@ -106,7 +106,7 @@ def test_select_ties_and_nans_bit_exact(seed):
         s[rng.random(s.shape) < 0.03] = np.inf
         s[rng.random(s.shape) < 0.05] = -0.0
         s[:, np.triu_indices(N, 1)[0], np.triu_indices(N, 1)[1]] = np.nan
-        packed.append(O.pack_causal(s))
+        packed.append(np.ascontiguousarray(O.pack_causal(s)))
         lists.append(O.select_all(s.astype(np.float64), O.tpd_plan(N, 0.3, 0.7)[2]))
     scores = torch.from_numpy(np.concatenate(packed, axis=1)).cuda()
     ws = S.workspace(prob)
