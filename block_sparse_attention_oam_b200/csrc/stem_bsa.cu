@@ -377,7 +377,9 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
       const int32_t* list;
       const int n = tile_len<DENSE>(p, tl, &list);
       if (n == 0) continue;
-      float m_run = -INFINITY, l_run = 0.f;
+      // l_run: sum of the rounded P the P.V product sees (normalises O);
+      // lt_run (FP8 only): sum of the unrounded P (gives the log-sum-exp)
+      float m_run = -INFINITY, l_run = 0.f, lt_run = 0.f;
       for (int jj = 0; jj < n; ++jj) {
         const uint32_t sb = is % 2, sph = (is / 2) & 1;
         if (!warp_wait(bar_s_full + 8 * sb, sph, abort_flag, p.status)) { alive = false; break; }
@@ -406,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
         // P = exp2(s * scale - m), written to the P buffer of this block (swizzled)
         const uint32_t pbuf = sP + (ipw % 2) * C::P_BYTES;
         ++ipw;
-        float sum = 0.f;
+        float sum = 0.f, sum_t = 0.f;
         if (!FP8) {
 #pragma unroll
           for (int u = 0; u < BN / 8; ++u) {
@@ -435,6 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
 #pragma unroll
               for (int q = 0; q < 4; ++q)
                 pv[q] = ex2_approx(fmaf(__uint_as_float(sr[16 * u + 4 * e + q]), p.scale_log2, -m_use));
+              sum_t += (pv[0] + pv[1]) + (pv[2] + pv[3]);
               const uint32_t lo = pack_e4m3x2(pv[0] * p.p_scale, pv[1] * p.p_scale);
               const uint32_t hi = pack_e4m3x2(pv[2] * p.p_scale, pv[3] * p.p_scale);
               w4[e] = lo | (hi << 16);
@@ -450,6 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
           }
         }
         l_run = l_run * alpha + sum;
+        if (FP8) lt_run = lt_run * alpha + sum_t;
         fence_proxy_async_smem();
         if (jj > 0) {
           // O holds the sum up to block jj-1 once its P V product is done
@@ -503,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
       }
       if (p.lse != nullptr && r < rows_valid)
         p.lse[static_cast<long long>(tl.h) * p.bt.total_tokens + tok] =
-            (m_run + __log2f(l_run / p.p_scale)) * 0.69314718055994531f;
+            (m_run + __log2f(FP8 ? lt_run : l_run)) * 0.69314718055994531f;
       tc_fence_before();
     }
   }
