@@ -203,6 +203,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default=W.LONG_128K_FP8.name, choices=sorted(W.ALL))
     ap.add_argument("--keep", type=float, default=None)
+    ap.add_argument("--seqlen", type=int, default=None, help="replace the workload's sequences by one of this length")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
@@ -211,6 +212,8 @@ def main():
     wl = W.ALL[args.workload]
     if args.keep is not None:
         wl = wl.with_(keep=args.keep)
+    if args.seqlen is not None:
+        wl = wl.with_(seqlens=(args.seqlen,), name=f"{wl.name}@{args.seqlen}")
     if args.impl == "reference":
         run_reference(args, wl)
         return
