@@ -350,6 +350,15 @@ stem_status_t check_qkv(const void* q, const void* k, const void* v, const stem_
 }
 
 }  // namespace
+
+stem_status_t set_last_error(stem_status_t s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
 }  // namespace stem
 
 using namespace stem;

@@ -279,6 +279,9 @@ __device__ __forceinline__ int tpd_k(double r, int N, double mu, int i) {
 
 #endif  // __CUDACC__
 
+// Record a message for stem_last_error() and return the status (host).
+stem_status_t set_last_error(stem_status_t s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+
 // ------------------------------------------------------------- host launchers
 struct PoolArgs {
   const void* x;            // contiguous [T, H, d] or paged cache [slots, P, H, d]

@@ -94,6 +94,7 @@ def lib() -> ctypes.CDLL:
         "bsa_prefill": ([pp, _P, _P, _P, pg, _P, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
         "bsa_dense_prefill": ([pp, _P, _P, _P, pg, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
         "stem_attention": ([pp, _P, _P, _P, pg, _P, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
+        "stem_attention_noalloc": ([pp, _P, _P, _P, pg, _P, _P, _P, _P, _P, _P], ctypes.c_int),
         "stem_query_status": ([_P, _P], ctypes.c_int),
         "stem_reset_status": ([_P, _P], ctypes.c_int),
         "stem_status_string": ([ctypes.c_int], ctypes.c_char_p),
@@ -250,6 +251,17 @@ def stem_attention(prob: Problem, q, k, v, paged: Optional[PagedKV] = None, out=
     ws = workspace(prob, q.device) if ws is None else ws
     _check(lib().stem_attention(prob.c, _ptr(q), _ptr(k), _ptr(v), _paged(paged), _ptr(out), _ptr(lse),
                                 _ptr(row_ptr), _ptr(col_idx), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def stem_attention_noalloc(prob: Problem, q, k, v, paged: Optional[PagedKV] = None, out=None, lse=None,
+                           row_ptr=None, col_idx=None, status=None, stream=None):
+    """stem_attention with the library's static scratch instead of a workspace
+    (for callers that cannot allocate device memory).  `status`: optional device
+    int32 tensor of one element that receives the call's device status word."""
+    out = _out(prob, q, out)
+    _check(lib().stem_attention_noalloc(prob.c, _ptr(q), _ptr(k), _ptr(v), _paged(paged), _ptr(out), _ptr(lse),
+                                        _ptr(row_ptr), _ptr(col_idx), _ptr(status), _stream(stream)))
     return out
 
 

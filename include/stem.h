@@ -178,6 +178,29 @@ STEM_API stem_status_t stem_attention(const stem_problem_t* prob, const void* q,
                              int32_t* col_idx_out, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * stem_attention without a caller workspace, for callers that cannot allocate
+ * device memory (a plugin or custom-operator host whose framework owns every
+ * byte of the GPU, a serving loop that must not allocate while it runs).  The
+ * paper has no counterpart: this is a deployment convenience of this library.
+ * Scratch comes from one fixed 32 MiB array compiled into the library, which
+ * every device that loads the library holds until the process exits; a problem
+ * whose stem_workspace_size() exceeds it is refused with STEM_ERR_WORKSPACE
+ * before anything is launched.  No call allocates or frees device memory.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current), so make that first call before any stream
+ * capture.  All calls on a device share the array and it keeps the last call's
+ * contents: calls that overlap on the GPU (other streams, other threads) race
+ * and must be serialised by the caller.  The status word is cleared at the start
+ * of each call; status_out (DEVICE uint32, or NULL) receives this call's device
+ * status word (0 = ok, bit 0 = pipeline wait timed out, bit 1 = bad block index).
+ * Other arguments as stem_attention.
+ */
+STEM_API stem_status_t stem_attention_noalloc(const stem_problem_t* prob, const void* q, const void* k,
+                                              const void* v, const stem_paged_kv_t* paged, void* out, float* lse,
+                                              int32_t* row_ptr_out, int32_t* col_idx_out, uint32_t* status_out,
+                                              void* stream);
+
+/*
  * Synchronise the stream, read and clear the device status word kept in the
  * workspace.  Returns STEM_OK, STEM_ERR_TIMEOUT, STEM_ERR_BOUNDS or STEM_ERR_CUDA.
  */
