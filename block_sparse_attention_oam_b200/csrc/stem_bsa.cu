@@ -7,22 +7,25 @@
 // being -inf, so the softmax stays exact; the inner path is the dense one.  The
 // same section notes native support for a paged KV cache.
 //
-// Design (one CTA per SM, persistent over (q-head, q-block) tiles, 6 warps):
-//   warp 0      TMA producer: Q tile once per tile, then K_j, V_j for every listed j
-//               into a 2-stage ring (64-row boxes, 128-byte swizzle; a paged cache
-//               is addressed page by page through the block table).
-//   warp 1      MMA issuer (one thread): S = Q K_j^T into one of two TMEM S buffers,
-//               then O += P_j V_j into the TMEM O accumulator.  S_{j+1} is issued
-//               before P_j is ready so the tensor core overlaps the softmax.
-//   warps 2..5  softmax (one thread per query row, TMEM lane quadrant = warp % 4):
-//               online softmax in the log2 domain, token-level causal mask on the
-//               diagonal block only (always the last list entry), lazy rescaling
-//               of O (only when the running max grows by more than 2^8), P written
-//               to shared memory for the P V product, then the epilogue (O / l ->
-//               bf16, log-sum-exp).
-// Every mbarrier wait is bounded (2 s); on expiry the CTA raises an abort flag,
-// records STEM_ERR_TIMEOUT in the status word, drains its tensor-core work and
-// releases its TMEM before exiting.
+// Design (one CTA per SM, persistent over (q-head, q-block) tiles, 10 warps):
+//   warp 0      TMA producer: the Q tile once per tile, then K_j and V_j of every listed
+//               block into separate rings (64-row boxes, 128-byte swizzle; a paged cache
+//               is read page by page through the block table).
+//   warp 1      MMA issuer (one thread): S = Q K_j^T into one of two TMEM S buffers, then
+//               O += P_j V_j with P read from TMEM (where the softmax wrote it over S_j)
+//               and V from shared memory.  S_{j+1} is issued before P_j is ready, so the
+//               tensor core overlaps the softmax.
+//   warps 2..9  softmax, two warpgroups: each query row is shared by two threads (one
+//               per warpgroup, half of the KV block's columns each); the row maximum is
+//               exchanged through shared memory once per block.  Online softmax in the
+//               log2 domain with packed fp32x2 arithmetic; the token-level causal mask is
+//               applied on the diagonal block only (always the last list entry); O is
+//               rescaled lazily (only when the running max grows by more than 2^8); O is
+//               normalised by the sum of the rounded P weights the product used; then
+//               the epilogue (O / l -> bf16, log-sum-exp).
+// Every wait is bounded (2 s); on expiry the CTA raises an abort flag, records
+// STEM_ERR_TIMEOUT in the status word, drains its tensor-core work, waits (bounded)
+// for its copies and releases its TMEM before exiting.
 #include <string.h>
 
 #include "stem_internal.cuh"
@@ -30,36 +33,46 @@
 namespace stem {
 namespace {
 
-constexpr int kBM = 128;         // query rows per tile (tcgen05 M)
-constexpr int kStages = 2;       // K/V ring depth
-constexpr int kThreads = 192;    // 6 warps
+constexpr int kBM = 128;              // query rows per tile (tcgen05 M)
+constexpr int kSoftmaxWarps = 8;
+constexpr int kThreads = 64 + 32 * kSoftmaxWarps;
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSmemCap = 227 * 1024;
 
 template <int D, int BN, bool FP8>
 struct Cfg {
   static constexpr int ES = FP8 ? 1 : 2;
   static constexpr int CH = 128 / ES;             // elements per 128-byte swizzle row
   static constexpr int DCH = D * ES / 128;        // 128-byte chunks along d
-  static constexpr int PCH = BN * ES / 128;       // 128-byte chunks along a P row
   static_assert(D * ES % 128 == 0 && BN * ES % 128 == 0, "rows must be whole 128-byte swizzle rows");
   static constexpr int Q_CHUNK = kBM * 128;
   static constexpr int KV_CHUNK = BN * 128;
   static constexpr int Q_BYTES = kBM * D * ES;
   static constexpr int KV_BYTES = BN * D * ES;
-  static constexpr int P_BYTES = kBM * BN * ES;
   static constexpr int S_KSTEPS = D * ES / 32;    // MMAs along d for S (32 bytes of K each)
   static constexpr int PV_KSTEPS = BN * ES / 32;  // MMAs along the KV block for O
   static constexpr int PV_KROWS = 32 / ES;        // KV rows consumed per PV MMA
   static constexpr int HALVES = BN / 64;          // 64-row TMA boxes per KV block
-  // shared memory carve-up (all tiles 1024-byte aligned for the 128-byte swizzle)
+  static constexpr int HALF = BN / 2;             // S columns per softmax thread
+  static constexpr int P_COLS = HALF * ES / 4;    // TMEM columns of one thread's P (packed)
+  static constexpr int O_HALF = D / 2;            // O columns per softmax thread
+  static constexpr int EXTRA = 512 + 2048 + 2048; // barriers, max exchange, sum exchange
+  static constexpr int SLACK = 1024;              // alignment of the tiles to 1024 bytes
+  // K / V ring depths: as deep as shared memory allows, at most 4
+  static constexpr int ROOM = static_cast<int>(kSmemCap) - Q_BYTES - EXTRA - SLACK;
+  static constexpr int KST = ROOM / KV_BYTES >= 8 ? 4 : (ROOM / KV_BYTES >= 6 ? 3 : 2);
+  static constexpr int VST = ROOM / KV_BYTES >= 8 ? 4 : (ROOM / KV_BYTES >= 5 ? (ROOM / KV_BYTES) - KST : 2);
+  static_assert(KST + VST <= ROOM / KV_BYTES, "K/V rings do not fit");
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + kStages * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + kStages * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
-  static constexpr int SMEM = OFF_BAR + 256 + 1024;  // + barriers + alignment slack
-  // force one CTA per SM (TMEM allocation takes all 512 columns)
+  static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
+  static constexpr int OFF_XMAX = OFF_BAR + 512;   // float [2 parity][2 wg][128]
+  static constexpr int OFF_XSUM = OFF_XMAX + 2048; // float [2 kind][2 wg][128]
+  static constexpr int SMEM = OFF_XSUM + 2048 + SLACK;
+  // force one CTA per SM (the TMEM allocation takes all 512 columns)
   static constexpr int SMEM_LAUNCH = SMEM < 120 * 1024 ? 120 * 1024 : SMEM;
+  static_assert(SMEM <= static_cast<int>(kSmemCap), "shared memory budget exceeded");
   static constexpr uint32_t FMT = FP8 ? 0u : 1u;  // e4m3 (kind::f8f6f4) or bf16 (kind::f16)
   static constexpr uint32_t IDESC_S = instr_desc(FMT, 0, 0, kBM, BN);
   static constexpr uint32_t IDESC_PV = instr_desc(FMT, 0, 1, kBM, D);
@@ -80,8 +93,9 @@ struct BsaParams {
   int Hq, Hkv;
   int total_tiles;
   float scale_log2;  // sigma * q_scale * k_scale * log2(e)
-  float out_scale;   // FP8: v_scale (l carries p_scale); BF16: 1
-  float p_scale;     // FP8: P is multiplied by this before rounding to e4m3
+  float p_bias;      // log2 of the factor P is scaled by before rounding (FP8: log2 1.75)
+  float out_scale;   // FP8: v_scale (l carries the P factor); BF16: 1
+  float p_scale;     // the factor itself (1 for BF16)
   uint32_t* status;
   signed char order[STEM_MAX_SEQS];  // sequences by decreasing block count
 };
@@ -108,7 +122,7 @@ __device__ __forceinline__ Tile decode_tile(const BsaParams& p, int t) {
   return r;
 }
 
-// Warp-uniform bounded wait on an mbarrier phase (see stem_internal.cuh).
+// Warp-uniform bounded wait on an mbarrier phase.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           uint32_t* status) {
   const unsigned full = 0xffffffffu;
@@ -153,39 +167,44 @@ template <int D, int BN, bool FP8, bool PAGED, bool DENSE>
 __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant__ BsaParams p) {
   using C = Cfg<D, BN, FP8>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sQ = sbase + C::OFF_Q;
   const uint32_t sK = sbase + C::OFF_K;
   const uint32_t sV = sbase + C::OFF_V;
-  const uint32_t sP = sbase + C::OFF_P;
   unsigned char* bar_area = smem + C::OFF_BAR;
+  float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX);
+  float* xsum = reinterpret_cast<float*>(smem + C::OFF_XSUM);
   // barriers (8 bytes each)
   const uint32_t b0 = sbase + C::OFF_BAR;
   const uint32_t bar_q_full = b0 + 0, bar_q_empty = b0 + 8;
-  const uint32_t bar_k_full = b0 + 16, bar_k_empty = b0 + 32;   // [2]
-  const uint32_t bar_v_full = b0 + 48, bar_v_empty = b0 + 64;   // [2]
-  const uint32_t bar_s_full = b0 + 80, bar_s_empty = b0 + 96;   // [2]
-  const uint32_t bar_p_full = b0 + 112, bar_pv_done = b0 + 120;
-  const uint32_t bar_drain = b0 + 128;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_area + 160);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 168);
+  const uint32_t bar_k_full = b0 + 16, bar_k_empty = b0 + 48;   // [4]
+  const uint32_t bar_v_full = b0 + 80, bar_v_empty = b0 + 112;  // [4]
+  const uint32_t bar_s_full = b0 + 144;                         // [2]
+  const uint32_t bar_p_full = b0 + 160, bar_pv_done = b0 + 168;
+  const uint32_t bar_drain = b0 + 176, bar_x = b0 + 184;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_area + 256);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 264);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (threadIdx.x == 0) {
     mbar_init(bar_q_full, 1);
     mbar_init(bar_q_empty, 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < C::KST; ++s) {
       mbar_init(bar_k_full + 8 * s, 1);
       mbar_init(bar_k_empty + 8 * s, 1);
+    }
+    for (int s = 0; s < C::VST; ++s) {
       mbar_init(bar_v_full + 8 * s, 1);
       mbar_init(bar_v_empty + 8 * s, 1);
-      mbar_init(bar_s_full + 8 * s, 1);
-      mbar_init(bar_s_empty + 8 * s, 4);
     }
-    mbar_init(bar_p_full, 4);
+    mbar_init(bar_s_full, 1);
+    mbar_init(bar_s_full + 8, 1);
+    mbar_init(bar_p_full, kSoftmaxWarps);
     mbar_init(bar_pv_done, 1);
     mbar_init(bar_drain, 1);
+    mbar_init(bar_x, kSoftmaxWarps);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -197,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_S = tmem;          // two buffers at columns 0 and 128
+  const uint32_t tmem_S = tmem;          // two buffers at columns 0 and 128 (P overwrites S)
   const uint32_t tmem_O = tmem + 256;    // D columns
 
   const int G = p.Hq / p.Hkv;
@@ -210,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
       tma_prefetch_map(&p.tk);
       tma_prefetch_map(&p.tv);
     }
-    uint32_t it = 0, tq = 0;
+    uint32_t itk = 0, itv = 0, tq = 0;
     bool alive = true;
     for (int t = blockIdx.x; t < p.total_tiles && alive; t += gridDim.x) {
       const Tile tl = decode_tile(p, t);
@@ -231,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
       ++tq;
       const int npages = (s.len + STEM_PAGE_SIZE - 1) / STEM_PAGE_SIZE;
       for (int j0 = 0; j0 < n && alive; j0 += 32) {
-        int jl = j0 + lane;
+        const int jl = j0 + lane;
         int myj = jl;
         if (!DENSE) myj = jl < n ? __ldg(list + jl) : 0;
         if (jl < n && (myj < 0 || myj > tl.i)) {
@@ -239,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
           myj = tl.i;
         }
         if (jl >= n) myj = 0;
-        // rows of this lane's block (one per 64-row half), resolved through the block table
+        // rows of this lane's block (one per 64-row box), resolved through the block table
         int rowh[C::HALVES];
 #pragma unroll
         for (int hh = 0; hh < C::HALVES; ++hh) {
@@ -261,64 +280,64 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
           int rows[C::HALVES];
 #pragma unroll
           for (int hh = 0; hh < C::HALVES; ++hh) rows[hh] = __shfl_sync(full, rowh[hh], q);
-          const uint32_t st = it % kStages, ph = (it / kStages) & 1;
-          if (!warp_wait(bar_k_empty + 8 * st, ph ^ 1, abort_flag, p.status)) { alive = false; break; }
+          const uint32_t ks = itk % C::KST, kph = (itk / C::KST) & 1;
+          if (!warp_wait(bar_k_empty + 8 * ks, kph ^ 1, abort_flag, p.status)) { alive = false; break; }
           if (lane == 0) {
-            mbar_arrive_expect_tx(bar_k_full + 8 * st, C::KV_BYTES);
+            mbar_arrive_expect_tx(bar_k_full + 8 * ks, C::KV_BYTES);
             for (int c = 0; c < C::DCH; ++c)
               for (int hh = 0; hh < C::HALVES; ++hh)
-                tma_load_3d(sK + st * C::KV_BYTES + c * C::KV_CHUNK + hh * 64 * 128, &p.tk, bar_k_full + 8 * st,
+                tma_load_3d(sK + ks * C::KV_BYTES + c * C::KV_CHUNK + hh * 64 * 128, &p.tk, bar_k_full + 8 * ks,
                             c * C::CH, kvh, rows[hh]);
           }
-          if (!warp_wait(bar_v_empty + 8 * st, ph ^ 1, abort_flag, p.status)) { alive = false; break; }
+          ++itk;
+          const uint32_t vs = itv % C::VST, vph = (itv / C::VST) & 1;
+          if (!warp_wait(bar_v_empty + 8 * vs, vph ^ 1, abort_flag, p.status)) { alive = false; break; }
           if (lane == 0) {
-            mbar_arrive_expect_tx(bar_v_full + 8 * st, C::KV_BYTES);
+            mbar_arrive_expect_tx(bar_v_full + 8 * vs, C::KV_BYTES);
             for (int c = 0; c < C::DCH; ++c)
               for (int hh = 0; hh < C::HALVES; ++hh)
-                tma_load_3d(sV + st * C::KV_BYTES + c * C::KV_CHUNK + hh * 64 * 128, &p.tv, bar_v_full + 8 * st,
+                tma_load_3d(sV + vs * C::KV_BYTES + c * C::KV_CHUNK + hh * 64 * 128, &p.tv, bar_v_full + 8 * vs,
                             c * C::CH, kvh, rows[hh]);
           }
-          ++it;
+          ++itv;
         }
       }
     }
     if (!alive) {
       // let the copies already issued land before the CTA can exit
-      for (uint32_t q = (it > kStages ? it - kStages : 0); q < it; ++q) {
-        const uint32_t st = q % kStages, ph = (q / kStages) & 1;
-        for (int spin = 0; spin < 1000000 && !mbar_try_wait(bar_k_full + 8 * st, ph); ++spin) {}
-        for (int spin = 0; spin < 1000000 && !mbar_try_wait(bar_v_full + 8 * st, ph); ++spin) {}
-      }
+      for (uint32_t q = (itk > C::KST ? itk - C::KST : 0); q < itk; ++q)
+        for (int spin = 0; spin < 1000000 && !mbar_try_wait(bar_k_full + 8 * (q % C::KST), (q / C::KST) & 1); ++spin) {}
+      for (uint32_t q = (itv > C::VST ? itv - C::VST : 0); q < itv; ++q)
+        for (int spin = 0; spin < 1000000 && !mbar_try_wait(bar_v_full + 8 * (q % C::VST), (q / C::VST) & 1); ++spin) {}
       if (tq > 0)
         for (int spin = 0; spin < 1000000 && !mbar_try_wait(bar_q_full, (tq - 1) & 1); ++spin) {}
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    uint32_t it_s = 0, it_v = 0, is = 0, ip = 0, tq = 0;
+    uint32_t itk = 0, itv = 0, is = 0, ip = 0, tq = 0;
     bool alive = true;
     auto issue_s = [&](void) -> bool {
-      const uint32_t sb = is % 2, sph = (is / 2) & 1;
-      const uint32_t st = it_s % kStages, kph = (it_s / kStages) & 1;
-      if (!warp_wait(bar_s_empty + 8 * sb, sph ^ 1, abort_flag, p.status)) return false;
-      if (!warp_wait(bar_k_full + 8 * st, kph, abort_flag, p.status)) return false;
+      const uint32_t sb = is % 2;
+      const uint32_t ks = itk % C::KST, kph = (itk / C::KST) & 1;
+      if (!warp_wait(bar_k_full + 8 * ks, kph, abort_flag, p.status)) return false;
       tc_fence_after();
       if (lane == 0) {
 #pragma unroll
-        for (int ks = 0; ks < C::S_KSTEPS; ++ks) {
-          const int c = ks / 4, w = ks % 4;
+        for (int k = 0; k < C::S_KSTEPS; ++k) {
+          const int c = k / 4, w = k % 4;
           const uint64_t ad = smem_desc_sw128(sQ + c * C::Q_CHUNK + w * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(sK + st * C::KV_BYTES + c * C::KV_CHUNK + w * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(sK + ks * C::KV_BYTES + c * C::KV_CHUNK + w * 32, 16, 1024);
           if (FP8)
-            mma_fp8(tmem_S + sb * 128, ad, bd, C::IDESC_S, ks > 0);
+            mma_fp8(tmem_S + sb * 128, ad, bd, C::IDESC_S, k > 0);
           else
-            mma_bf16(tmem_S + sb * 128, ad, bd, C::IDESC_S, ks > 0);
+            mma_bf16(tmem_S + sb * 128, ad, bd, C::IDESC_S, k > 0);
         }
         mma_commit(bar_s_full + 8 * sb);
-        mma_commit(bar_k_empty + 8 * st);
+        mma_commit(bar_k_empty + 8 * ks);
       }
       __syncwarp();
       ++is;
-      ++it_s;
+      ++itk;
       return true;
     };
     for (int t = blockIdx.x; t < p.total_tiles && alive; t += gridDim.x) {
@@ -340,25 +359,25 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
         const uint32_t pb = ip % 2;
         if (!warp_wait(bar_p_full, ip & 1, abort_flag, p.status)) { alive = false; break; }
         ++ip;
-        const uint32_t st = it_v % kStages, vph = (it_v / kStages) & 1;
-        if (!warp_wait(bar_v_full + 8 * st, vph, abort_flag, p.status)) { alive = false; break; }
+        const uint32_t vs = itv % C::VST, vph = (itv / C::VST) & 1;
+        if (!warp_wait(bar_v_full + 8 * vs, vph, abort_flag, p.status)) { alive = false; break; }
         tc_fence_after();
         if (lane == 0) {
 #pragma unroll
-          for (int ks = 0; ks < C::PV_KSTEPS; ++ks) {
-            const int c = (ks * 32) / 128, w = ks % 4;
-            const uint64_t ad = smem_desc_sw128(sP + pb * C::P_BYTES + c * C::Q_CHUNK + w * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(sV + st * C::KV_BYTES + ks * C::PV_KROWS * 128, C::KV_CHUNK, 1024);
+          for (int k = 0; k < C::PV_KSTEPS; ++k) {
+            const uint64_t bd =
+                smem_desc_sw128(sV + vs * C::KV_BYTES + k * C::PV_KROWS * 128, C::KV_CHUNK, 1024);
+            const uint32_t acc = (jj > 0 || k > 0) ? 1u : 0u;
             if (FP8)
-              mma_fp8(tmem_O, ad, bd, C::IDESC_PV, (jj > 0 || ks > 0) ? 1u : 0u);
+              mma_fp8_ts(tmem_O, tmem_S + pb * 128 + k * 8, bd, C::IDESC_PV, acc);
             else
-              mma_bf16(tmem_O, ad, bd, C::IDESC_PV, (jj > 0 || ks > 0) ? 1u : 0u);
+              mma_bf16_ts(tmem_O, tmem_S + pb * 128 + k * 8, bd, C::IDESC_PV, acc);
           }
-          mma_commit(bar_v_empty + 8 * st);
+          mma_commit(bar_v_empty + 8 * vs);
           mma_commit(bar_pv_done);
         }
         __syncwarp();
-        ++it_v;
+        ++itv;
       }
     }
     // drain: every tcgen05.mma issued by this thread has completed
@@ -367,94 +386,110 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
     for (int spin = 0; spin < 4000000 && !mbar_try_wait(bar_drain, 0); ++spin) {}
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    const int quad = warp % 4;
+    const int wg = (warp - 2) / 4;                   // which half of the KV block's columns
+    const int quad = warp % 4;                       // TMEM lane quadrant of this warp
     const int r = quad * 32 + lane;                  // query row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    uint32_t is = 0, ipv = 0, ipw = 0;
+    const float sl2 = p.scale_log2;
+    uint32_t is = 0, ipv = 0, ix = 0;
     bool alive = true;
+    // exchange through shared memory: write mine, meet the other warpgroup, read theirs
+    auto exchange = [&](float* buf, float mine) -> float {
+      buf[wg * 128 + r] = mine;
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence_block();
+        mbar_arrive(bar_x);
+      }
+      const bool ok = warp_wait(bar_x, ix & 1, abort_flag, p.status);
+      ++ix;
+      if (!ok) {
+        alive = false;
+        return 0.f;
+      }
+      return buf[(1 - wg) * 128 + r];
+    };
     for (int t = blockIdx.x; t < p.total_tiles && alive; t += gridDim.x) {
       const Tile tl = decode_tile(p, t);
       const int32_t* list;
       const int n = tile_len<DENSE>(p, tl, &list);
       if (n == 0) continue;
-      // l_run: sum of the rounded P the P.V product sees (normalises O);
-      // lt_run (FP8 only): sum of the unrounded P (gives the log-sum-exp)
-      float m_run = -INFINITY, l_run = 0.f, lt_run = 0.f;
+      // l: sum of the rounded P the product uses (normalises O); lt (FP8): unrounded sum (LSE)
+      float m_run = -INFINITY;
+      float2 l2 = make_float2(0.f, 0.f), lt2 = make_float2(0.f, 0.f);
       for (int jj = 0; jj < n; ++jj) {
         const uint32_t sb = is % 2, sph = (is / 2) & 1;
         if (!warp_wait(bar_s_full + 8 * sb, sph, abort_flag, p.status)) { alive = false; break; }
         ++is;
         tc_fence_after();
-        uint32_t sr[BN];
+        uint32_t sr[C::HALF];
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) tmem_ld32(tmem_S + sb * 128 + lane_off + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+        for (int c = 0; c < C::HALF / 16; ++c) tmem_ld16(tmem_S + sb * 128 + wg * C::HALF + lane_off + c * 16, &sr[c * 16]);
         tmem_wait_ld();
         tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_s_empty + 8 * sb);
         const bool diag = (jj == n - 1);
         float mx = -INFINITY;
+        if (diag) {
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          float v = __uint_as_float(sr[c]);
-          if (diag && c > r) v = -INFINITY;
-          sr[c] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
+          for (int c = 0; c < C::HALF; ++c)
+            if (wg * C::HALF + c > r) sr[c] = __float_as_uint(-INFINITY);
         }
-        const float m_new = fmaxf(m_run, mx * p.scale_log2);
+#pragma unroll
+        for (int c = 0; c < C::HALF; c += 2) mx = max3f(mx, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+        const float other = exchange(xmax + (jj & 1) * 256, mx);
+        if (!alive) break;
+        tc_fence_after();
+        const float m_new = max3f(m_run, mx * sl2, other * sl2);
         const bool resc = m_new > m_run + 8.0f;
         const float m_use = resc ? m_new : m_run;
         const float alpha = resc ? ex2_approx(m_run - m_use) : 1.0f;
-        // P = exp2(s * scale - m), written to the P buffer of this block (swizzled)
-        const uint32_t pbuf = sP + (ipw % 2) * C::P_BYTES;
-        ++ipw;
-        float sum = 0.f, sum_t = 0.f;
+        const float2 sc2 = make_float2(sl2, sl2);
+        const float2 bias2 = make_float2(p.p_bias - m_use, p.p_bias - m_use);
+        float2 sum2 = make_float2(0.f, 0.f), sumt2 = make_float2(0.f, 0.f);
+        uint32_t pk[C::P_COLS];
         if (!FP8) {
 #pragma unroll
-          for (int u = 0; u < BN / 8; ++u) {
-            uint32_t w4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float p0 = ex2_approx(fmaf(__uint_as_float(sr[8 * u + 2 * e]), p.scale_log2, -m_use));
-              const float p1 = ex2_approx(fmaf(__uint_as_float(sr[8 * u + 2 * e + 1]), p.scale_log2, -m_use));
-              w4[e] = pack_bf16x2(p0, p1);
-              // normalise with the rounded weights the P.V product uses
-              sum += __uint_as_float(w4[e] << 16) + __uint_as_float(w4[e] & 0xFFFF0000u);
-            }
-            const int chunk = u / 8, uu = u % 8;
-            const uint32_t addr = pbuf + chunk * C::Q_CHUNK + r * 128 + ((uu ^ (r & 7)) << 4);
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w4[0]), "r"(w4[1]), "r"(w4[2]),
-                         "r"(w4[3])
-                         : "memory");
+          for (int u = 0; u < C::HALF / 2; ++u) {
+            const float2 y = fma2(make_float2(__uint_as_float(sr[2 * u]), __uint_as_float(sr[2 * u + 1])), sc2, bias2);
+            const uint32_t w = pack_bf16x2(ex2_approx(y.x), ex2_approx(y.y));
+            pk[u] = w;
+            sum2 = add2(sum2, make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
           }
         } else {
 #pragma unroll
-          for (int u = 0; u < BN / 16; ++u) {
-            uint32_t w4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float pv[4];
-#pragma unroll
-              for (int q = 0; q < 4; ++q)
-                pv[q] = ex2_approx(fmaf(__uint_as_float(sr[16 * u + 4 * e + q]), p.scale_log2, -m_use));
-              sum_t += (pv[0] + pv[1]) + (pv[2] + pv[3]);
-              const uint32_t lo = pack_e4m3x2(pv[0] * p.p_scale, pv[1] * p.p_scale);
-              const uint32_t hi = pack_e4m3x2(pv[2] * p.p_scale, pv[3] * p.p_scale);
-              w4[e] = lo | (hi << 16);
-              // normalise with the rounded (scaled) weights the P.V product uses
-              const float2 a = e4m3x2_to_float2(static_cast<uint16_t>(lo));
-              const float2 b = e4m3x2_to_float2(static_cast<uint16_t>(hi));
-              sum += (a.x + a.y) + (b.x + b.y);
-            }
-            const uint32_t addr = pbuf + r * 128 + ((u ^ (r & 7)) << 4);
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w4[0]), "r"(w4[1]), "r"(w4[2]),
-                         "r"(w4[3])
-                         : "memory");
+          for (int u = 0; u < C::HALF / 4; ++u) {
+            const float2 y0 = fma2(make_float2(__uint_as_float(sr[4 * u]), __uint_as_float(sr[4 * u + 1])), sc2, bias2);
+            const float2 y1 = fma2(make_float2(__uint_as_float(sr[4 * u + 2]), __uint_as_float(sr[4 * u + 3])), sc2, bias2);
+            const float2 e0 = make_float2(ex2_approx(y0.x), ex2_approx(y0.y));
+            const float2 e1 = make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
+            const uint32_t lo = pack_e4m3x2(e0.x, e0.y);
+            const uint32_t hi = pack_e4m3x2(e1.x, e1.y);
+            pk[u] = lo | (hi << 16);
+            sum2 = add2(sum2, add2(e4m3x2_to_float2(static_cast<uint16_t>(lo)),
+                                   e4m3x2_to_float2(static_cast<uint16_t>(hi))));
+            sumt2 = add2(sumt2, add2(e0, e1));
           }
         }
-        l_run = l_run * alpha + sum;
-        if (FP8) lt_run = lt_run * alpha + sum_t;
-        fence_proxy_async_smem();
+        // P overwrites this thread's half of the S buffer, packed along columns
+        if (C::P_COLS == 32) {
+          tmem_st16(tmem_S + sb * 128 + wg * C::P_COLS + lane_off, &pk[0]);
+          tmem_st16(tmem_S + sb * 128 + wg * C::P_COLS + lane_off + 16, &pk[16]);
+        } else if (C::P_COLS == 16) {
+          tmem_st16(tmem_S + sb * 128 + wg * C::P_COLS + lane_off, &pk[0]);
+        } else {
+          uint32_t tmp[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) tmp[e] = e < C::P_COLS ? pk[e % C::P_COLS] : 0u;
+          static_assert(C::P_COLS == 32 || C::P_COLS == 16 || C::P_COLS == 8, "P columns");
+          asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
+                           tmem_S + sb * 128 + wg * C::P_COLS + lane_off),
+                       "r"(tmp[0]), "r"(tmp[1]), "r"(tmp[2]), "r"(tmp[3]), "r"(tmp[4]), "r"(tmp[5]), "r"(tmp[6]),
+                       "r"(tmp[7])
+                       : "memory");
+        }
+        const float2 a2 = make_float2(alpha, alpha);
+        l2 = fma2(l2, a2, sum2);
+        if (FP8) lt2 = fma2(lt2, a2, sumt2);
         if (jj > 0) {
           // O holds the sum up to block jj-1 once its P V product is done
           if (!warp_wait(bar_pv_done, ipv & 1, abort_flag, p.status)) { alive = false; break; }
@@ -462,52 +497,66 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
           tc_fence_after();
           if (__any_sync(full, resc)) {
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t o[32];
-              tmem_ld32(tmem_O + lane_off + c * 32, o);
+            for (int c = 0; c < C::O_HALF / 16; ++c) {
+              uint32_t o[16];
+              const uint32_t addr = tmem_O + wg * C::O_HALF + lane_off + c * 16;
+              tmem_ld16(addr, o);
               tmem_wait_ld();
 #pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st32(tmem_O + lane_off + c * 32, o);
+              for (int e = 0; e < 16; e += 2) {
+                const float2 v = mul2(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2);
+                o[e] = __float_as_uint(v.x);
+                o[e + 1] = __float_as_uint(v.y);
+              }
+              tmem_st16(addr, o);
             }
-            tmem_wait_st();
           }
         }
+        tmem_wait_st();
         m_run = m_use;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_p_full);
       }
       if (!alive) break;
-      // epilogue: wait for the last P V product, normalise, store
+      // epilogue: wait for the last P V product, combine the halves' sums, normalise, store
       if (!warp_wait(bar_pv_done, ipv & 1, abort_flag, p.status)) { alive = false; break; }
       ++ipv;
       tc_fence_after();
+      const float l_mine = l2.x + l2.y;
+      const float l = l_mine + exchange(xsum, l_mine);
+      if (!alive) break;
+      float lt = l;
+      if (FP8) {
+        const float lt_mine = lt2.x + lt2.y;
+        lt = lt_mine + exchange(xsum + 256, lt_mine);
+        if (!alive) break;
+      }
       const SeqInfo& s = p.bt.seq[tl.b];
       const int rows_valid = min(BN, s.len - tl.i * BN);
-      const float inv = p.out_scale / l_run;
+      const float inv = p.out_scale / l;
       const long long tok = static_cast<long long>(s.tok0) + tl.i * BN + r;
-      unsigned char* orow = static_cast<unsigned char*>(p.out) + (tok * p.Hq + tl.h) * D * 2;
+      unsigned char* orow = static_cast<unsigned char*>(p.out) + ((tok * p.Hq + tl.h) * D + wg * C::O_HALF) * 2;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tmem_O + lane_off + c * 32, o);
+      for (int c = 0; c < C::O_HALF / 16; ++c) {
+        uint32_t o[16];
+        tmem_ld16(tmem_O + wg * C::O_HALF + lane_off + c * 16, o);
         tmem_wait_ld();
         if (r < rows_valid) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+          for (int q = 0; q < 2; ++q) {
             uint4 v;
             v.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv, __uint_as_float(o[8 * q + 1]) * inv);
             v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv);
             v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv);
             v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + (c * 32 + 8 * q) * 2) = v;
+            *reinterpret_cast<uint4*>(orow + (c * 16 + 8 * q) * 2) = v;
           }
         }
       }
-      if (p.lse != nullptr && r < rows_valid)
+      if (p.lse != nullptr && wg == 0 && r < rows_valid)
         p.lse[static_cast<long long>(tl.h) * p.bt.total_tokens + tok] =
-            (m_run + __log2f(FP8 ? lt_run : l_run)) * 0.69314718055994531f;
+            (m_run + __log2f(FP8 ? lt / p.p_scale : lt)) * 0.69314718055994531f;
       tc_fence_before();
     }
   }
@@ -599,6 +648,7 @@ cudaError_t launch_bsa(const Batch& bt, const BsaArgs& a, bool fp8, bool paged, 
   prm.scale_log2 = a.sigma * (fp8 ? a.q_scale * a.k_scale : 1.0f) * log2e;
   // FP8: P <= 2^8 after the lazy max update; 448 / 256 keeps it inside e4m3's range.
   prm.p_scale = fp8 ? 1.75f : 1.0f;
+  prm.p_bias = fp8 ? 0.80735492205760410f : 0.0f;  // log2(1.75)
   // l is accumulated from the scaled, rounded P, so the V scale is all that remains
   prm.out_scale = fp8 ? a.v_scale : 1.0f;
   long long tiles = 0;
