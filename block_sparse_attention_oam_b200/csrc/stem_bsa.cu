@@ -15,14 +15,15 @@
 //               O += P_j V_j with P read from TMEM (where the softmax wrote it over S_j)
 //               and V from shared memory.  S_{j+1} is issued before P_j is ready, so the
 //               tensor core overlaps the softmax.
-//   warps 2..9  softmax, two warpgroups: each query row is shared by two threads (one
-//               per warpgroup, half of the KV block's columns each); the row maximum is
-//               exchanged through shared memory once per block.  Online softmax in the
-//               log2 domain with packed fp32x2 arithmetic; the token-level causal mask is
-//               applied on the diagonal block only (always the last list entry); O is
-//               rescaled lazily (only when the running max grows by more than 2^8); O is
-//               normalised by the sum of the rounded P weights the product used; then
-//               the epilogue (O / l -> bf16, log-sum-exp).
+//   warps 2..9  softmax, two warpgroups: each query row is shared by two threads, one per
+//               warpgroup, each owning half of every KV block's columns.  The halves run
+//               independent online softmaxes (own running max, own sum, own O accumulator
+//               in TMEM) and are merged once per tile in the epilogue, so no per-block
+//               exchange between them is needed.  Log2 domain, packed fp32x2 arithmetic;
+//               the token-level causal mask only on the diagonal block (always the last
+//               list entry); lazy rescaling of O (only when a running max grows by more
+//               than 2^8), waiting for the previous P V product only then; O normalised
+//               by the sum of the rounded P weights the product used.
 // Every wait is bounded (2 s); on expiry the CTA raises an abort flag, records
 // STEM_ERR_TIMEOUT in the status word, drains its tensor-core work, waits (bounded)
 // for its copies and releases its TMEM before exiting.
@@ -55,8 +56,9 @@ struct Cfg {
   static constexpr int HALVES = BN / 64;          // 64-row TMA boxes per KV block
   static constexpr int HALF = BN / 2;             // S columns per softmax thread
   static constexpr int P_COLS = HALF * ES / 4;    // TMEM columns of one thread's P (packed)
-  static constexpr int O_HALF = D / 2;            // O columns per softmax thread
-  static constexpr int EXTRA = 512 + 2048 + 2048; // barriers, max exchange, sum exchange
+  static constexpr int O_HALF = D / 2;            // output columns stored per softmax thread
+  static constexpr int PV_HSTEPS = PV_KSTEPS / 2; // P V MMAs per half (one O accumulator each)
+  static constexpr int EXTRA = 512 + 3072;        // barriers, per-tile (m, l, lt) exchange
   static constexpr int SLACK = 1024;              // alignment of the tiles to 1024 bytes
   // K / V ring depths: as deep as shared memory allows, at most 4
   static constexpr int ROOM = static_cast<int>(kSmemCap) - Q_BYTES - EXTRA - SLACK;
@@ -67,9 +69,8 @@ struct Cfg {
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
-  static constexpr int OFF_XMAX = OFF_BAR + 512;   // float [2 parity][2 wg][128]
-  static constexpr int OFF_XSUM = OFF_XMAX + 2048; // float [2 kind][2 wg][128]
-  static constexpr int SMEM = OFF_XSUM + 2048 + SLACK;
+  static constexpr int OFF_XCH = OFF_BAR + 512;    // float [3 kind][2 wg][128]
+  static constexpr int SMEM = OFF_XCH + 3072 + SLACK;
   // force one CTA per SM (the TMEM allocation takes all 512 columns)
   static constexpr int SMEM_LAUNCH = SMEM < 120 * 1024 ? 120 * 1024 : SMEM;
   static_assert(SMEM <= static_cast<int>(kSmemCap), "shared memory budget exceeded");
@@ -174,8 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
   const uint32_t sK = sbase + C::OFF_K;
   const uint32_t sV = sbase + C::OFF_V;
   unsigned char* bar_area = smem + C::OFF_BAR;
-  float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX);
-  float* xsum = reinterpret_cast<float*>(smem + C::OFF_XSUM);
+  float* xch = reinterpret_cast<float*>(smem + C::OFF_XCH);
   // barriers (8 bytes each)
   const uint32_t b0 = sbase + C::OFF_BAR;
   const uint32_t bar_q_full = b0 + 0, bar_q_empty = b0 + 8;
@@ -216,8 +216,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_S = tmem;          // two buffers at columns 0 and 128 (P overwrites S)
-  const uint32_t tmem_O = tmem + 256;    // D columns
+  const uint32_t tmem_S = tmem;          // two S buffers at columns 0 and 128 (P overwrites S)
+  const uint32_t tmem_O = tmem + 256;    // O of half 0 at 256, of half 1 at 256 + D
 
   const int G = p.Hq / p.Hkv;
   const unsigned full = 0xffffffffu;
@@ -365,13 +365,17 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
         if (lane == 0) {
 #pragma unroll
           for (int k = 0; k < C::PV_KSTEPS; ++k) {
+            // half hf of the block's keys: its P (in that half's S columns) into its own O
+            const int hf = k / C::PV_HSTEPS, kk = k % C::PV_HSTEPS;
             const uint64_t bd =
                 smem_desc_sw128(sV + vs * C::KV_BYTES + k * C::PV_KROWS * 128, C::KV_CHUNK, 1024);
-            const uint32_t acc = (jj > 0 || k > 0) ? 1u : 0u;
+            const uint32_t a_tmem = tmem_S + pb * 128 + hf * C::HALF + kk * 8;
+            const uint32_t d_tmem = tmem_O + hf * D;
+            const uint32_t acc = (jj > 0 || kk > 0) ? 1u : 0u;
             if (FP8)
-              mma_fp8_ts(tmem_O, tmem_S + pb * 128 + k * 8, bd, C::IDESC_PV, acc);
+              mma_fp8_ts(d_tmem, a_tmem, bd, C::IDESC_PV, acc);
             else
-              mma_bf16_ts(tmem_O, tmem_S + pb * 128 + k * 8, bd, C::IDESC_PV, acc);
+              mma_bf16_ts(d_tmem, a_tmem, bd, C::IDESC_PV, acc);
           }
           mma_commit(bar_v_empty + 8 * vs);
           mma_commit(bar_pv_done);
@@ -390,56 +394,38 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
     const int quad = warp % 4;                       // TMEM lane quadrant of this warp
     const int r = quad * 32 + lane;                  // query row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t my_O = tmem_O + wg * D + lane_off;
     const float sl2 = p.scale_log2;
-    uint32_t is = 0, ipv = 0, ix = 0;
+    uint32_t gb = 0, ix = 0;                         // blocks processed by this CTA; exchanges
     bool alive = true;
-    // exchange through shared memory: write mine, meet the other warpgroup, read theirs
-    auto exchange = [&](float* buf, float mine) -> float {
-      buf[wg * 128 + r] = mine;
-      __syncwarp();
-      if (lane == 0) {
-        __threadfence_block();
-        mbar_arrive(bar_x);
-      }
-      const bool ok = warp_wait(bar_x, ix & 1, abort_flag, p.status);
-      ++ix;
-      if (!ok) {
-        alive = false;
-        return 0.f;
-      }
-      return buf[(1 - wg) * 128 + r];
-    };
     for (int t = blockIdx.x; t < p.total_tiles && alive; t += gridDim.x) {
       const Tile tl = decode_tile(p, t);
       const int32_t* list;
       const int n = tile_len<DENSE>(p, tl, &list);
       if (n == 0) continue;
-      // l: sum of the rounded P the product uses (normalises O); lt (FP8): unrounded sum (LSE)
+      // per half: running max, sum of the rounded P the product uses (normalises O) and,
+      // for FP8, the sum of the unrounded P (log-sum-exp)
       float m_run = -INFINITY;
       float2 l2 = make_float2(0.f, 0.f), lt2 = make_float2(0.f, 0.f);
-      for (int jj = 0; jj < n; ++jj) {
-        const uint32_t sb = is % 2, sph = (is / 2) & 1;
+      for (int jj = 0; jj < n; ++jj, ++gb) {
+        const uint32_t sb = gb % 2, sph = (gb / 2) & 1;
         if (!warp_wait(bar_s_full + 8 * sb, sph, abort_flag, p.status)) { alive = false; break; }
-        ++is;
         tc_fence_after();
+        const uint32_t my_S = tmem_S + sb * 128 + wg * C::HALF + lane_off;
         uint32_t sr[C::HALF];
 #pragma unroll
-        for (int c = 0; c < C::HALF / 16; ++c) tmem_ld16(tmem_S + sb * 128 + wg * C::HALF + lane_off + c * 16, &sr[c * 16]);
+        for (int c = 0; c < C::HALF / 16; ++c) tmem_ld16(my_S + c * 16, &sr[c * 16]);
         tmem_wait_ld();
-        tc_fence_before();
         const bool diag = (jj == n - 1);
-        float mx = -INFINITY;
         if (diag) {
 #pragma unroll
           for (int c = 0; c < C::HALF; ++c)
             if (wg * C::HALF + c > r) sr[c] = __float_as_uint(-INFINITY);
         }
+        float mx = -INFINITY;
 #pragma unroll
         for (int c = 0; c < C::HALF; c += 2) mx = max3f(mx, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
-        const float other = exchange(xmax + (jj & 1) * 256, mx);
-        if (!alive) break;
-        tc_fence_after();
-        const float m_new = max3f(m_run, mx * sl2, other * sl2);
+        const float m_new = fmaxf(m_run, mx * sl2);
         const bool resc = m_new > m_run + 8.0f;
         const float m_use = resc ? m_new : m_run;
         const float alpha = resc ? ex2_approx(m_run - m_use) : 1.0f;
@@ -470,46 +456,30 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
             sumt2 = add2(sumt2, add2(e0, e1));
           }
         }
-        // P overwrites this thread's half of the S buffer, packed along columns
-        if (C::P_COLS == 32) {
-          tmem_st16(tmem_S + sb * 128 + wg * C::P_COLS + lane_off, &pk[0]);
-          tmem_st16(tmem_S + sb * 128 + wg * C::P_COLS + lane_off + 16, &pk[16]);
-        } else if (C::P_COLS == 16) {
-          tmem_st16(tmem_S + sb * 128 + wg * C::P_COLS + lane_off, &pk[0]);
-        } else {
-          uint32_t tmp[16];
+        // P overwrites the first columns of this half's S, packed along columns
+        static_assert(C::P_COLS == 32 || C::P_COLS == 16, "P columns per half");
 #pragma unroll
-          for (int e = 0; e < 16; ++e) tmp[e] = e < C::P_COLS ? pk[e % C::P_COLS] : 0u;
-          static_assert(C::P_COLS == 32 || C::P_COLS == 16 || C::P_COLS == 8, "P columns");
-          asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
-                           tmem_S + sb * 128 + wg * C::P_COLS + lane_off),
-                       "r"(tmp[0]), "r"(tmp[1]), "r"(tmp[2]), "r"(tmp[3]), "r"(tmp[4]), "r"(tmp[5]), "r"(tmp[6]),
-                       "r"(tmp[7])
-                       : "memory");
-        }
+        for (int c = 0; c < C::P_COLS / 16; ++c) tmem_st16(my_S + c * 16, &pk[c * 16]);
         const float2 a2 = make_float2(alpha, alpha);
         l2 = fma2(l2, a2, sum2);
         if (FP8) lt2 = fma2(lt2, a2, sumt2);
-        if (jj > 0) {
-          // O holds the sum up to block jj-1 once its P V product is done
-          if (!warp_wait(bar_pv_done, ipv & 1, abort_flag, p.status)) { alive = false; break; }
-          ++ipv;
+        if (jj > 0 && __any_sync(full, resc)) {
+          // O of this half holds the sum up to the previous block once its P V product is
+          // done (the barrier cannot be two phases ahead: the next product needs this warp)
+          if (!warp_wait(bar_pv_done, (gb - 1) & 1, abort_flag, p.status)) { alive = false; break; }
           tc_fence_after();
-          if (__any_sync(full, resc)) {
 #pragma unroll
-            for (int c = 0; c < C::O_HALF / 16; ++c) {
-              uint32_t o[16];
-              const uint32_t addr = tmem_O + wg * C::O_HALF + lane_off + c * 16;
-              tmem_ld16(addr, o);
-              tmem_wait_ld();
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t o[16];
+            tmem_ld16(my_O + c * 16, o);
+            tmem_wait_ld();
 #pragma unroll
-              for (int e = 0; e < 16; e += 2) {
-                const float2 v = mul2(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2);
-                o[e] = __float_as_uint(v.x);
-                o[e + 1] = __float_as_uint(v.y);
-              }
-              tmem_st16(addr, o);
+            for (int e = 0; e < 16; e += 2) {
+              const float2 v = mul2(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2);
+              o[e] = __float_as_uint(v.x);
+              o[e + 1] = __float_as_uint(v.y);
             }
+            tmem_st16(my_O + c * 16, o);
           }
         }
         tmem_wait_st();
@@ -519,44 +489,55 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
         if (lane == 0) mbar_arrive(bar_p_full);
       }
       if (!alive) break;
-      // epilogue: wait for the last P V product, combine the halves' sums, normalise, store
-      if (!warp_wait(bar_pv_done, ipv & 1, abort_flag, p.status)) { alive = false; break; }
-      ++ipv;
+      // epilogue: wait for the last P V product, merge the two halves, normalise, store
+      if (!warp_wait(bar_pv_done, (gb - 1) & 1, abort_flag, p.status)) { alive = false; break; }
       tc_fence_after();
-      const float l_mine = l2.x + l2.y;
-      const float l = l_mine + exchange(xsum, l_mine);
-      if (!alive) break;
-      float lt = l;
-      if (FP8) {
-        const float lt_mine = lt2.x + lt2.y;
-        lt = lt_mine + exchange(xsum + 256, lt_mine);
-        if (!alive) break;
+      float* mine = xch + wg * 128 + r;
+      mine[0] = m_run;
+      mine[256] = l2.x + l2.y;
+      mine[512] = lt2.x + lt2.y;
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence_block();
+        mbar_arrive(bar_x);
       }
+      if (!warp_wait(bar_x, ix & 1, abort_flag, p.status)) { alive = false; break; }
+      ++ix;
+      const float m0 = xch[r], m1 = xch[128 + r];
+      const float l0 = xch[256 + r], l1 = xch[384 + r];
+      const float t0 = xch[512 + r], t1 = xch[640 + r];
+      const float mf = fmaxf(m0, m1);
+      const float f0 = ex2_approx(m0 - mf), f1 = ex2_approx(m1 - mf);
+      const float l = l0 * f0 + l1 * f1;
+      const float inv = p.out_scale / l;
+      const float g0 = f0 * inv, g1 = f1 * inv;
       const SeqInfo& s = p.bt.seq[tl.b];
       const int rows_valid = min(BN, s.len - tl.i * BN);
-      const float inv = p.out_scale / l;
       const long long tok = static_cast<long long>(s.tok0) + tl.i * BN + r;
       unsigned char* orow = static_cast<unsigned char*>(p.out) + ((tok * p.Hq + tl.h) * D + wg * C::O_HALF) * 2;
+      const float2 gg0 = make_float2(g0, g0), gg1 = make_float2(g1, g1);
 #pragma unroll
       for (int c = 0; c < C::O_HALF / 16; ++c) {
-        uint32_t o[16];
-        tmem_ld16(tmem_O + wg * C::O_HALF + lane_off + c * 16, o);
+        uint32_t oa[16], ob[16];
+        tmem_ld16(tmem_O + wg * C::O_HALF + lane_off + c * 16, oa);
+        tmem_ld16(tmem_O + D + wg * C::O_HALF + lane_off + c * 16, ob);
         tmem_wait_ld();
         if (r < rows_valid) {
+          uint32_t w[8];
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv, __uint_as_float(o[8 * q + 1]) * inv);
-            v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv);
-            v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv);
-            v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + (c * 16 + 8 * q) * 2) = v;
+          for (int e = 0; e < 16; e += 2) {
+            const float2 v = fma2(make_float2(__uint_as_float(oa[e]), __uint_as_float(oa[e + 1])), gg0,
+                                  mul2(make_float2(__uint_as_float(ob[e]), __uint_as_float(ob[e + 1])), gg1));
+            w[e / 2] = pack_bf16x2(v.x, v.y);
           }
+          *reinterpret_cast<uint4*>(orow + c * 32) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(orow + c * 32 + 16) = make_uint4(w[4], w[5], w[6], w[7]);
         }
       }
-      if (p.lse != nullptr && wg == 0 && r < rows_valid)
-        p.lse[static_cast<long long>(tl.h) * p.bt.total_tokens + tok] =
-            (m_run + __log2f(FP8 ? lt / p.p_scale : lt)) * 0.69314718055994531f;
+      if (p.lse != nullptr && wg == 0 && r < rows_valid) {
+        const float lt = FP8 ? (t0 * f0 + t1 * f1) / p.p_scale : l;
+        p.lse[static_cast<long long>(tl.h) * p.bt.total_tokens + tok] = (mf + __log2f(lt)) * 0.69314718055994531f;
+      }
       tc_fence_before();
     }
   }
