@@ -430,7 +430,9 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
         const float m_use = resc ? m_new : m_run;
         const float alpha = resc ? ex2_approx(m_run - m_use) : 1.0f;
         const float2 sc2 = make_float2(sl2, sl2);
-        const float2 bias2 = make_float2(p.p_bias - m_use, p.p_bias - m_use);
+        // a half that has seen only masked keys so far (m = -inf) gets P = 0, not NaN
+        const float m_sub = m_use == -INFINITY ? 0.f : m_use;
+        const float2 bias2 = make_float2(p.p_bias - m_sub, p.p_bias - m_sub);
         float2 sum2 = make_float2(0.f, 0.f), sumt2 = make_float2(0.f, 0.f);
         uint32_t pk[C::P_COLS];
         if (!FP8) {
