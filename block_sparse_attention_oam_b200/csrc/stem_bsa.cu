@@ -105,17 +105,24 @@ struct Tile {
   int b, i, h;
 };
 
+// Tile order: sequences by decreasing length; inside a sequence kv-head by kv-head, rows
+// from the last (longest list) to the first, the g q-heads of a row adjacent.  The CTAs
+// running at one time then share one kv-head's K/V, which fits in L2.
 __device__ __forceinline__ Tile decode_tile(const BsaParams& p, int t) {
   Tile r{0, 0, 0};
+  const int G = p.Hq / p.Hkv;
   int acc = 0;
   for (int q = 0; q < p.bt.num_seqs; ++q) {
     const int b = p.order[q];
-    const int nt = p.bt.seq[b].nblk * p.Hq;
+    const int nb = p.bt.seq[b].nblk;
+    const int nt = nb * p.Hq;
     if (t < acc + nt) {
       const int local = t - acc;
+      const int kvh = local / (nb * G);
+      const int rem = local - kvh * nb * G;
       r.b = b;
-      r.i = p.bt.seq[b].nblk - 1 - local / p.Hq;
-      r.h = local % p.Hq;
+      r.i = nb - 1 - rem / G;
+      r.h = kvh * G + rem % G;
       return r;
     }
     acc += nt;
@@ -127,15 +134,12 @@ __device__ __forceinline__ Tile decode_tile(const BsaParams& p, int t) {
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           uint32_t* status) {
   const unsigned full = 0xffffffffu;
-  int spins = 0;
-  uint64_t t0 = 0;
-  for (;;) {
-    const bool ok = mbar_try_wait(bar, parity);
-    if (__all_sync(full, ok)) return true;
-    const int ab = __shfl_sync(full, *abort_flag, 0);
-    if (ab) return false;
-    if (++spins == 8) t0 = global_ns();
-    if (spins > 8) {
+  if (__all_sync(full, mbar_try_wait(bar, parity))) return true;
+  uint64_t t0 = global_ns();
+  for (int spins = 1;; ++spins) {
+    if (__all_sync(full, mbar_try_wait(bar, parity))) return true;
+    if ((spins & 31) == 0) {
+      if (__shfl_sync(full, *abort_flag, 0)) return false;
       const bool late = __shfl_sync(full, (global_ns() - t0) > kWaitLimitNs ? 1 : 0, 0);
       if (late) {
         if ((threadIdx.x & 31) == 0) {
@@ -414,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
         const uint32_t my_S = tmem_S + sb * 128 + wg * C::HALF + lane_off;
         uint32_t sr[C::HALF];
 #pragma unroll
-        for (int c = 0; c < C::HALF / 16; ++c) tmem_ld16(my_S + c * 16, &sr[c * 16]);
+        for (int c = 0; c < C::HALF / 32; ++c) tmem_ld32(my_S + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
         tmem_wait_ld();
         const bool diag = (jj == n - 1);
         if (diag) {
@@ -422,9 +426,13 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
           for (int c = 0; c < C::HALF; ++c)
             if (wg * C::HALF + c > r) sr[c] = __float_as_uint(-INFINITY);
         }
-        float mx = -INFINITY;
+        // row maximum with four independent chains
+        float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < C::HALF; c += 2) mx = max3f(mx, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+        for (int c = 0; c < C::HALF; c += 8)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) mq[q] = max3f(mq[q], __uint_as_float(sr[c + 2 * q]), __uint_as_float(sr[c + 2 * q + 1]));
+        const float mx = fmaxf(max3f(mq[0], mq[1], mq[2]), mq[3]);
         const float m_new = fmaxf(m_run, mx * sl2);
         const bool resc = m_new > m_run + 8.0f;
         const float m_use = resc ? m_new : m_run;
@@ -433,7 +441,13 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
         // a half that has seen only masked keys so far (m = -inf) gets P = 0, not NaN
         const float m_sub = m_use == -INFINITY ? 0.f : m_use;
         const float2 bias2 = make_float2(p.p_bias - m_sub, p.p_bias - m_sub);
-        float2 sum2 = make_float2(0.f, 0.f), sumt2 = make_float2(0.f, 0.f);
+        // sums with four independent chains
+        float2 sq[4], tq4[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          sq[q] = make_float2(0.f, 0.f);
+          tq4[q] = make_float2(0.f, 0.f);
+        }
         uint32_t pk[C::P_COLS];
         if (!FP8) {
 #pragma unroll
@@ -441,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
             const float2 y = fma2(make_float2(__uint_as_float(sr[2 * u]), __uint_as_float(sr[2 * u + 1])), sc2, bias2);
             const uint32_t w = pack_bf16x2(ex2_approx(y.x), ex2_approx(y.y));
             pk[u] = w;
-            sum2 = add2(sum2, make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
+            sq[u % 4] = add2(sq[u % 4], make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
           }
         } else {
 #pragma unroll
@@ -453,15 +467,19 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
             const uint32_t lo = pack_e4m3x2(e0.x, e0.y);
             const uint32_t hi = pack_e4m3x2(e1.x, e1.y);
             pk[u] = lo | (hi << 16);
-            sum2 = add2(sum2, add2(e4m3x2_to_float2(static_cast<uint16_t>(lo)),
-                                   e4m3x2_to_float2(static_cast<uint16_t>(hi))));
-            sumt2 = add2(sumt2, add2(e0, e1));
+            sq[u % 4] = add2(sq[u % 4], add2(e4m3x2_to_float2(static_cast<uint16_t>(lo)),
+                                             e4m3x2_to_float2(static_cast<uint16_t>(hi))));
+            tq4[u % 4] = add2(tq4[u % 4], add2(e0, e1));
           }
         }
+        const float2 sum2 = add2(add2(sq[0], sq[1]), add2(sq[2], sq[3]));
+        const float2 sumt2 = add2(add2(tq4[0], tq4[1]), add2(tq4[2], tq4[3]));
         // P overwrites the first columns of this half's S, packed along columns
         static_assert(C::P_COLS == 32 || C::P_COLS == 16, "P columns per half");
-#pragma unroll
-        for (int c = 0; c < C::P_COLS / 16; ++c) tmem_st16(my_S + c * 16, &pk[c * 16]);
+        if constexpr (C::P_COLS == 32)
+          tmem_st32(my_S, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+        else
+          tmem_st16(my_S, &pk[0]);
         const float2 a2 = make_float2(alpha, alpha);
         l2 = fma2(l2, a2, sum2);
         if (FP8) lt2 = fma2(lt2, a2, sumt2);
