@@ -15,21 +15,21 @@
 //               O += P_j V_j with P read from TMEM (where the softmax wrote it over S_j)
 //               and V from shared memory.  S_{j+1} is issued before P_j is ready, so the
 //               tensor core overlaps the softmax.
-//   warps 2..17 softmax, four warpgroups: each query row is shared by four threads,
-//               one per warpgroup, each owning a quarter of every KV block's columns (four
-//               warps per SM sub-partition hide the MUFU and TMEM latencies).  The two
-//               quarters of a half exchange their partial row maximum through shared
-//               memory once per block; each half runs its own online softmax into its own
-//               O accumulator in TMEM, and the halves are merged once per tile in the
-//               epilogue.  Log2 domain, packed fp32x2 arithmetic; the token-level causal
-//               mask only on the diagonal block (always the last list entry); lazy
-//               rescaling of O (only when a running max grows by more than 2^8), waiting
-//               for the previous P V product only then; O normalised by the sum of the
-//               rounded P weights the product used.
+//   warps 2..9  softmax, two warpgroups: each query row is shared by two threads, one per
+//               warpgroup, each owning half of every KV block's columns.  The halves run
+//               independent online softmaxes (own running max, own sum, own O accumulator
+//               in TMEM) and are merged once per tile in the epilogue, so no per-block
+//               exchange between them is needed.  Log2 domain, packed fp32x2 arithmetic;
+//               the token-level causal mask only on the diagonal block (always the last
+//               list entry); lazy rescaling of O (only when a running max grows by more
+//               than 2^8), waiting for the previous P V product only then; O normalised
+//               by the sum of the rounded P weights the product used.
 // Every wait is bounded (2 s); on expiry the CTA raises an abort flag, records
 // STEM_ERR_TIMEOUT in the status word, drains its tensor-core work, waits (bounded)
 // for its copies and releases its TMEM before exiting.
 #include <string.h>
+
+#include <type_traits>
 
 #include "stem_internal.cuh"
 
@@ -37,7 +37,7 @@ namespace stem {
 namespace {
 
 constexpr int kBM = 128;              // query rows per tile (tcgen05 M)
-constexpr int kSoftmaxWarps = 16;
+constexpr int kSoftmaxWarps = 8;
 constexpr int kThreads = 64 + 32 * kSoftmaxWarps;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSmemCap = 227 * 1024;
@@ -56,12 +56,11 @@ struct Cfg {
   static constexpr int PV_KSTEPS = BN * ES / 32;  // MMAs along the KV block for O
   static constexpr int PV_KROWS = 32 / ES;        // KV rows consumed per PV MMA
   static constexpr int HALVES = BN / 64;          // 64-row TMA boxes per KV block
-  static constexpr int HALF = BN / 2;             // S columns of one half (one O accumulator)
-  static constexpr int PART = BN / 4;             // S columns per softmax thread
-  static constexpr int P_COLS = PART * ES / 4;    // TMEM columns of one thread's P (packed)
-  static constexpr int O_PART = D / 4;            // output columns stored per softmax thread
-  static constexpr int PV_HSTEPS = PV_KSTEPS / 2; // P V MMAs per half
-  static constexpr int EXTRA = 512 + 4096 + 6144; // barriers, max exchange, per-tile exchange
+  static constexpr int HALF = BN / 2;             // S columns per softmax thread
+  static constexpr int P_COLS = HALF * ES / 4;    // TMEM columns of one thread's P (packed)
+  static constexpr int O_HALF = D / 2;            // output columns stored per softmax thread
+  static constexpr int PV_HSTEPS = PV_KSTEPS / 2; // P V MMAs per half (one O accumulator each)
+  static constexpr int EXTRA = 512 + 3072;        // barriers, per-tile (m, l, lt) exchange
   static constexpr int SLACK = 1024;              // alignment of the tiles to 1024 bytes
   // K / V ring depths: as deep as shared memory allows, at most 4
   static constexpr int ROOM = static_cast<int>(kSmemCap) - Q_BYTES - EXTRA - SLACK;
@@ -72,9 +71,8 @@ struct Cfg {
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
-  static constexpr int OFF_XMAX = OFF_BAR + 512;   // float [2 parity][4 part][128]
-  static constexpr int OFF_XCH = OFF_XMAX + 4096;  // float [3 kind][4 part][128]
-  static constexpr int SMEM = OFF_XCH + 6144 + SLACK;
+  static constexpr int OFF_XCH = OFF_BAR + 512;    // float [3 kind][2 wg][128]
+  static constexpr int SMEM = OFF_XCH + 3072 + SLACK;
   // force one CTA per SM (the TMEM allocation takes all 512 columns)
   static constexpr int SMEM_LAUNCH = SMEM < 120 * 1024 ? 120 * 1024 : SMEM;
   static_assert(SMEM <= static_cast<int>(kSmemCap), "shared memory budget exceeded");
@@ -183,7 +181,6 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
   const uint32_t sK = sbase + C::OFF_K;
   const uint32_t sV = sbase + C::OFF_V;
   unsigned char* bar_area = smem + C::OFF_BAR;
-  float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX);
   float* xch = reinterpret_cast<float*>(smem + C::OFF_XCH);
   // barriers (8 bytes each)
   const uint32_t b0 = sbase + C::OFF_BAR;
@@ -193,9 +190,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
   const uint32_t bar_s_full = b0 + 144;                         // [2]
   const uint32_t bar_p_full = b0 + 160, bar_pv_done = b0 + 168;
   const uint32_t bar_drain = b0 + 176, bar_x = b0 + 184;
-  const uint32_t bar_pair = b0 + 192;                            // [8]: (half, lane quadrant)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_area + 320);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 328);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_area + 256);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 264);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (threadIdx.x == 0) {
@@ -215,7 +211,6 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
     mbar_init(bar_pv_done, 1);
     mbar_init(bar_drain, 1);
     mbar_init(bar_x, kSoftmaxWarps);
-    for (int q = 0; q < 8; ++q) mbar_init(bar_pair + 8 * q, 2);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -401,68 +396,52 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
     for (int spin = 0; spin < 4000000 && !mbar_try_wait(bar_drain, 0); ++spin) {}
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    const int part = (warp - 2) / 4;                 // which quarter of the KV block's columns
-    const int half = part / 2, sub = part % 2;       // O accumulator, position within the half
+    const int wg = (warp - 2) / 4;                   // which half of the KV block's columns
     const int quad = warp % 4;                       // TMEM lane quadrant of this warp
     const int r = quad * 32 + lane;                  // query row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t my_O = tmem_O + half * D + sub * (D / 2) + lane_off;   // this thread's rescale range
-    const uint32_t my_pair = bar_pair + 8 * (half * 4 + quad);
+    const uint32_t my_O = tmem_O + wg * D + lane_off;
     const float sl2 = p.scale_log2;
-    uint32_t gb = 0, ix = 0, ipair = 0;              // blocks processed; tile and pair exchanges
+    uint32_t gb = 0, ix = 0;                         // blocks processed by this CTA; exchanges
     bool alive = true;
     for (int t = blockIdx.x; t < p.total_tiles && alive; t += gridDim.x) {
       const Tile tl = decode_tile(p, t);
       const int32_t* list;
       const int n = tile_len<DENSE>(p, tl, &list);
       if (n == 0) continue;
-      // per half: running max (shared by its two quarters), and per thread the partial sums
-      // of the rounded P the product uses (normalise O) and, for FP8, of the unrounded P (LSE)
+      // per half: running max, sum of the rounded P the product uses (normalises O) and,
+      // for FP8, the sum of the unrounded P (log-sum-exp)
       float m_run = -INFINITY;
       float2 l2 = make_float2(0.f, 0.f), lt2 = make_float2(0.f, 0.f);
       for (int jj = 0; jj < n; ++jj, ++gb) {
         const uint32_t sb = gb % 2, sph = (gb / 2) & 1;
         if (!warp_wait(bar_s_full + 8 * sb, sph, abort_flag, p.status)) { alive = false; break; }
         tc_fence_after();
-        const uint32_t my_S = tmem_S + sb * 128 + part * C::PART + lane_off;
-        uint32_t sr[C::PART];
-        if constexpr (C::PART == 32)
-          tmem_ld32(my_S, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        else
-          tmem_ld16(my_S, &sr[0]);
+        const uint32_t my_S = tmem_S + sb * 128 + wg * C::HALF + lane_off;
+        uint32_t sr[C::HALF];
+#pragma unroll
+        for (int c = 0; c < C::HALF / 32; ++c) tmem_ld32(my_S + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
         tmem_wait_ld();
-        tc_fence_before();
         const bool diag = (jj == n - 1);
         if (diag) {
 #pragma unroll
-          for (int c = 0; c < C::PART; ++c)
-            if (part * C::PART + c > r) sr[c] = __float_as_uint(-INFINITY);
+          for (int c = 0; c < C::HALF; ++c)
+            if (wg * C::HALF + c > r) sr[c] = __float_as_uint(-INFINITY);
         }
-        // partial row maximum (four independent chains), then the partner quarter's
+        // row maximum with four independent chains
         float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < C::PART; c += 8)
+        for (int c = 0; c < C::HALF; c += 8)
 #pragma unroll
           for (int q = 0; q < 4; ++q) mq[q] = max3f(mq[q], __uint_as_float(sr[c + 2 * q]), __uint_as_float(sr[c + 2 * q + 1]));
-        const float mx_mine = fmaxf(max3f(mq[0], mq[1], mq[2]), mq[3]);
-        float* xm = xmax + (gb & 1) * 512;
-        xm[part * 128 + r] = mx_mine;
-        __syncwarp();
-        if (lane == 0) {
-          __threadfence_block();
-          mbar_arrive(my_pair);
-        }
-        if (!warp_wait(my_pair, ipair & 1, abort_flag, p.status)) { alive = false; break; }
-        ++ipair;
-        tc_fence_after();
-        const float mx = fmaxf(mx_mine, xm[(part ^ 1) * 128 + r]);
+        const float mx = fmaxf(max3f(mq[0], mq[1], mq[2]), mq[3]);
         const float m_new = fmaxf(m_run, mx * sl2);
         const bool resc = m_new > m_run + 8.0f;
         const float m_use = resc ? m_new : m_run;
         const float alpha = resc ? ex2_approx(m_run - m_use) : 1.0f;
+        const float2 sc2 = make_float2(sl2, sl2);
         // a half that has seen only masked keys so far (m = -inf) gets P = 0, not NaN
         const float m_sub = m_use == -INFINITY ? 0.f : m_use;
-        const float2 sc2 = make_float2(sl2, sl2);
         const float2 bias2 = make_float2(p.p_bias - m_sub, p.p_bias - m_sub);
         // sums with four independent chains
         float2 sq[4], tq4[4];
@@ -474,47 +453,52 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
         uint32_t pk[C::P_COLS];
         if (!FP8) {
 #pragma unroll
-          for (int u = 0; u < C::PART / 2; ++u) {
+          for (int u = 0; u < C::HALF / 2; ++u) {
             const float2 y = fma2(make_float2(__uint_as_float(sr[2 * u]), __uint_as_float(sr[2 * u + 1])), sc2, bias2);
             const uint32_t w = pack_bf16x2(ex2_approx(y.x), ex2_approx(y.y));
             pk[u] = w;
             sq[u % 4] = add2(sq[u % 4], make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
           }
         } else {
+          // e4m3 P; its rounded values are summed as f16 pairs (exact enough: two e4m3
+          // codes per f16 add) and the unrounded values only when the LSE is requested
+          auto fp8_block = [&](auto want_lse) {
 #pragma unroll
-          for (int u = 0; u < C::PART / 4; ++u) {
-            const float2 y0 = fma2(make_float2(__uint_as_float(sr[4 * u]), __uint_as_float(sr[4 * u + 1])), sc2, bias2);
-            const float2 y1 = fma2(make_float2(__uint_as_float(sr[4 * u + 2]), __uint_as_float(sr[4 * u + 3])), sc2, bias2);
-            const float2 e0 = make_float2(ex2_approx(y0.x), ex2_approx(y0.y));
-            const float2 e1 = make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
-            const uint32_t lo = pack_e4m3x2(e0.x, e0.y);
-            const uint32_t hi = pack_e4m3x2(e1.x, e1.y);
-            pk[u] = lo | (hi << 16);
-            sq[u % 4] = add2(sq[u % 4], add2(e4m3x2_to_float2(static_cast<uint16_t>(lo)),
-                                             e4m3x2_to_float2(static_cast<uint16_t>(hi))));
-            tq4[u % 4] = add2(tq4[u % 4], add2(e0, e1));
-          }
+            for (int u = 0; u < C::HALF / 4; ++u) {
+              const float2 y0 = fma2(make_float2(__uint_as_float(sr[4 * u]), __uint_as_float(sr[4 * u + 1])), sc2, bias2);
+              const float2 y1 = fma2(make_float2(__uint_as_float(sr[4 * u + 2]), __uint_as_float(sr[4 * u + 3])), sc2, bias2);
+              const float2 e0 = make_float2(ex2_approx(y0.x), ex2_approx(y0.y));
+              const float2 e1 = make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
+              const uint32_t lo = pack_e4m3x2(e0.x, e0.y);
+              const uint32_t hi = pack_e4m3x2(e1.x, e1.y);
+              pk[u] = __byte_perm(lo, hi, 0x5410);
+              sq[u % 4] = add2(sq[u % 4], e4m3x4_pairsum(pk[u]));
+              if constexpr (decltype(want_lse)::value) tq4[u % 4] = add2(tq4[u % 4], add2(e0, e1));
+            }
+          };
+          if (p.lse != nullptr)
+            fp8_block(std::true_type{});
+          else
+            fp8_block(std::false_type{});
         }
         const float2 sum2 = add2(add2(sq[0], sq[1]), add2(sq[2], sq[3]));
         const float2 sumt2 = add2(add2(tq4[0], tq4[1]), add2(tq4[2], tq4[3]));
-        // P of this quarter, packed along columns, into its half's P range (the partner's
-        // S columns may be overwritten: both quarters have read S before the exchange)
-        const uint32_t my_P = tmem_S + sb * 128 + half * C::HALF + sub * C::P_COLS + lane_off;
-        static_assert(C::P_COLS == 16 || C::P_COLS == 8, "P columns per quarter");
-        if constexpr (C::P_COLS == 16)
-          tmem_st16(my_P, &pk[0]);
+        // P overwrites the first columns of this half's S, packed along columns
+        static_assert(C::P_COLS == 32 || C::P_COLS == 16, "P columns per half");
+        if constexpr (C::P_COLS == 32)
+          tmem_st32(my_S, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
         else
-          tmem_st8(my_P, &pk[0]);
+          tmem_st16(my_S, &pk[0]);
         const float2 a2 = make_float2(alpha, alpha);
         l2 = fma2(l2, a2, sum2);
         if (FP8) lt2 = fma2(lt2, a2, sumt2);
         if (jj > 0 && __any_sync(full, resc)) {
-          // this half's O holds the sum up to the previous block once its P V product is
+          // O of this half holds the sum up to the previous block once its P V product is
           // done (the barrier cannot be two phases ahead: the next product needs this warp)
           if (!warp_wait(bar_pv_done, (gb - 1) & 1, abort_flag, p.status)) { alive = false; break; }
           tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < D / 16; ++c) {
             uint32_t o[16];
             tmem_ld16(my_O + c * 16, o);
             tmem_wait_ld();
@@ -537,10 +521,10 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
       // epilogue: wait for the last P V product, merge the two halves, normalise, store
       if (!warp_wait(bar_pv_done, (gb - 1) & 1, abort_flag, p.status)) { alive = false; break; }
       tc_fence_after();
-      float* mine = xch + part * 128 + r;
+      float* mine = xch + wg * 128 + r;
       mine[0] = m_run;
-      mine[512] = l2.x + l2.y;
-      mine[1024] = lt2.x + lt2.y;
+      mine[256] = l2.x + l2.y;
+      mine[512] = lt2.x + lt2.y;
       __syncwarp();
       if (lane == 0) {
         __threadfence_block();
@@ -548,9 +532,9 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
       }
       if (!warp_wait(bar_x, ix & 1, abort_flag, p.status)) { alive = false; break; }
       ++ix;
-      const float m0 = xch[r], m1 = xch[256 + r];                       // half 0 = parts 0,1; half 1 = 2,3
-      const float l0 = xch[512 + r] + xch[640 + r], l1 = xch[768 + r] + xch[896 + r];
-      const float t0 = xch[1024 + r] + xch[1152 + r], t1 = xch[1280 + r] + xch[1408 + r];
+      const float m0 = xch[r], m1 = xch[128 + r];
+      const float l0 = xch[256 + r], l1 = xch[384 + r];
+      const float t0 = xch[512 + r], t1 = xch[640 + r];
       const float mf = fmaxf(m0, m1);
       const float f0 = ex2_approx(m0 - mf), f1 = ex2_approx(m1 - mf);
       const float l = l0 * f0 + l1 * f1;
@@ -559,13 +543,13 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
       const SeqInfo& s = p.bt.seq[tl.b];
       const int rows_valid = min(BN, s.len - tl.i * BN);
       const long long tok = static_cast<long long>(s.tok0) + tl.i * BN + r;
-      unsigned char* orow = static_cast<unsigned char*>(p.out) + ((tok * p.Hq + tl.h) * D + part * C::O_PART) * 2;
+      unsigned char* orow = static_cast<unsigned char*>(p.out) + ((tok * p.Hq + tl.h) * D + wg * C::O_HALF) * 2;
       const float2 gg0 = make_float2(g0, g0), gg1 = make_float2(g1, g1);
 #pragma unroll
-      for (int c = 0; c < C::O_PART / 16; ++c) {
+      for (int c = 0; c < C::O_HALF / 16; ++c) {
         uint32_t oa[16], ob[16];
-        tmem_ld16(tmem_O + part * C::O_PART + lane_off + c * 16, oa);
-        tmem_ld16(tmem_O + D + part * C::O_PART + lane_off + c * 16, ob);
+        tmem_ld16(tmem_O + wg * C::O_HALF + lane_off + c * 16, oa);
+        tmem_ld16(tmem_O + D + wg * C::O_HALF + lane_off + c * 16, ob);
         tmem_wait_ld();
         if (r < rows_valid) {
           uint32_t w[8];
@@ -579,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
           *reinterpret_cast<uint4*>(orow + c * 32 + 16) = make_uint4(w[4], w[5], w[6], w[7]);
         }
       }
-      if (p.lse != nullptr && part == 0 && r < rows_valid) {
+      if (p.lse != nullptr && wg == 0 && r < rows_valid) {
         const float lt = FP8 ? (t0 * f0 + t1 * f1) / p.p_scale : l;
         p.lse[static_cast<long long>(tl.h) * p.bt.total_tokens + tok] = (mf + __log2f(lt)) * 0.69314718055994531f;
       }

@@ -331,6 +331,19 @@ __device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t v) {
   return make_float2(lo, hi);
 }
 
+// Four e4m3 codes (bytes 0..3) -> (b0 + b2, b1 + b3) as floats, the pair sums taken in f16.
+__device__ __forceinline__ float2 e4m3x4_pairsum(uint32_t v) {
+  uint32_t a, b, c;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(a) : "h"(static_cast<uint16_t>(v & 0xFFFFu)));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(b) : "h"(static_cast<uint16_t>(v >> 16)));
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(c) : "r"(a), "r"(b));
+  float lo, hi;
+  asm("{\n\t.reg .f16 x, y;\n\tmov.b32 {x, y}, %2;\n\tcvt.f32.f16 %0, x;\n\tcvt.f32.f16 %1, y;\n\t}\n"
+      : "=f"(lo), "=f"(hi)
+      : "r"(c));
+  return make_float2(lo, hi);
+}
+
 // Locate the sequence owning a global block row.
 __device__ __forceinline__ int seq_of_row(const Batch& bt, int row) {
   int b = 0;
