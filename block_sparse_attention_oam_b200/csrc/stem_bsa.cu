@@ -451,44 +451,35 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
           tq4[q] = make_float2(0.f, 0.f);
         }
         uint32_t pk[C::P_COLS];
-        // exponentials: MUFU for most pairs, the FMA-pipe polynomial for NPOLY of every 8
-        // (groups of pairs / quads), never on the diagonal block (masked keys must give 0)
-        auto exps = [&](auto npoly_c, auto want_lse) {
-          constexpr int NPOLY = decltype(npoly_c)::value;
-          if constexpr (!FP8) {
+        if (!FP8) {
 #pragma unroll
-            for (int u = 0; u < C::HALF / 2; ++u) {
-              const float2 y = fma2(make_float2(__uint_as_float(sr[2 * u]), __uint_as_float(sr[2 * u + 1])), sc2, bias2);
-              const float2 e = (u % 8) < NPOLY ? exp2_poly<3>(y) : make_float2(ex2_approx(y.x), ex2_approx(y.y));
-              const uint32_t w = pack_bf16x2(e.x, e.y);
-              pk[u] = w;
-              sq[u % 4] = add2(sq[u % 4], make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
-            }
-          } else {
-            // e4m3 P; its rounded values are summed as f16 pairs (exact enough: two e4m3
-            // codes per f16 add) and the unrounded values only when the LSE is requested
+          for (int u = 0; u < C::HALF / 2; ++u) {
+            const float2 y = fma2(make_float2(__uint_as_float(sr[2 * u]), __uint_as_float(sr[2 * u + 1])), sc2, bias2);
+            const uint32_t w = pack_bf16x2(ex2_approx(y.x), ex2_approx(y.y));
+            pk[u] = w;
+            sq[u % 4] = add2(sq[u % 4], make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
+          }
+        } else {
+          // e4m3 P; its rounded values are summed as f16 pairs (exact enough: two e4m3
+          // codes per f16 add) and the unrounded values only when the LSE is requested
+          auto fp8_block = [&](auto want_lse) {
 #pragma unroll
             for (int u = 0; u < C::HALF / 4; ++u) {
               const float2 y0 = fma2(make_float2(__uint_as_float(sr[4 * u]), __uint_as_float(sr[4 * u + 1])), sc2, bias2);
               const float2 y1 = fma2(make_float2(__uint_as_float(sr[4 * u + 2]), __uint_as_float(sr[4 * u + 3])), sc2, bias2);
-              const bool poly = (u % 8) < NPOLY;
-              const float2 e0 = poly ? exp2_poly<2>(y0) : make_float2(ex2_approx(y0.x), ex2_approx(y0.y));
-              const float2 e1 = poly ? exp2_poly<2>(y1) : make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
+              const float2 e0 = make_float2(ex2_approx(y0.x), ex2_approx(y0.y));
+              const float2 e1 = make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
               const uint32_t lo = pack_e4m3x2(e0.x, e0.y);
               const uint32_t hi = pack_e4m3x2(e1.x, e1.y);
               pk[u] = __byte_perm(lo, hi, 0x5410);
               sq[u % 4] = add2(sq[u % 4], e4m3x4_pairsum(pk[u]));
               if constexpr (decltype(want_lse)::value) tq4[u % 4] = add2(tq4[u % 4], add2(e0, e1));
             }
-          }
-        };
-        constexpr int kPoly = FP8 ? 4 : 3;
-        if (diag) {
-          if (FP8 && p.lse != nullptr) exps(std::integral_constant<int, 0>{}, std::true_type{});
-          else exps(std::integral_constant<int, 0>{}, std::false_type{});
-        } else {
-          if (FP8 && p.lse != nullptr) exps(std::integral_constant<int, kPoly>{}, std::true_type{});
-          else exps(std::integral_constant<int, kPoly>{}, std::false_type{});
+          };
+          if (p.lse != nullptr)
+            fp8_block(std::true_type{});
+          else
+            fp8_block(std::false_type{});
         }
         const float2 sum2 = add2(add2(sq[0], sq[1]), add2(sq[2], sq[3]));
         const float2 sumt2 = add2(add2(tq4[0], tq4[1]), add2(tq4[2], tq4[3]));

@@ -331,34 +331,6 @@ __device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t v) {
   return make_float2(lo, hi);
 }
 
-// 2^y for a pair on the FMA pipe, to share the exponential load with the MUFU unit.
-// Cody-Waite reduction y = j + f with j the nearest integer (adding 1.5 * 2^23 rounds
-// to an integer) and f in [-1/2, 1/2]; 2^f from a minimax polynomial fitted here by the
-// Remez exchange (max relative error 7.5e-5 for degree 3, 1.7e-3 for degree 2); j is
-// added to the exponent field.  y is clamped to -125 (the result stays a normal float,
-// below 2^-124); callers use the MUFU ex2 wherever an exact 0 for -inf is needed.
-template <int DEG>
-__device__ __forceinline__ float2 exp2_poly(float2 y) {
-  const float magic = 12582912.0f;
-  y.x = fmaxf(y.x, -125.f);
-  y.y = fmaxf(y.y, -125.f);
-  const float2 t = add2(y, make_float2(magic, magic));
-  const float2 jf = add2(t, make_float2(-magic, -magic));
-  const float2 f = fma2(jf, make_float2(-1.f, -1.f), y);
-  float2 p;
-  if (DEG == 3) {
-    p = fma2(make_float2(0.0551716685f, 0.0551716685f), f, make_float2(0.242611125f, 0.242611125f));
-    p = fma2(p, f, make_float2(0.693260968f, 0.693260968f));
-    p = fma2(p, f, make_float2(0.999928057f, 0.999928057f));
-  } else {
-    p = fma2(make_float2(0.238428935f, 0.238428935f), f, make_float2(0.703447998f, 0.703447998f));
-    p = fma2(p, f, make_float2(1.00044310f, 1.00044310f));
-  }
-  // low 9 bits of t's pattern hold j (two's complement); shifted they add j to the exponent
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
-}
-
 // Four e4m3 codes (bytes 0..3) -> (b0 + b2, b1 + b3) as floats, the pair sums taken in f16.
 __device__ __forceinline__ float2 e4m3x4_pairsum(uint32_t v) {
   uint32_t a, b, c;
