@@ -196,6 +196,60 @@ def run_reference(args, wl):
     print(json.dumps(line), flush=True)
 
 
+def run_sweep(args):
+    """Density sweep: BSA latency against the selected FLOPs for several keep
+    fractions on one workload, next to the dense kernel (the pages report the
+    latency as close to linear in density)."""
+    wl = W.ALL[args.workload] if args.workload != W.LONG_128K_FP8.name else W.SWEEP_64K
+    inp = W.make_inputs(wl)
+    q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
+    stream = torch.cuda.current_stream()
+    rows = []
+    dense_ms = None
+    for keep in W.SWEEP_KEEPS:
+        prob = S.problem_for(wl.with_(keep=keep), inp)
+        sz = prob.sizes()
+        ws = S.workspace(prob)
+        scores = torch.empty((wl.num_q_heads, sz["scores_per_head"]), dtype=torch.float32, device="cuda")
+        rp = torch.empty(sz["num_rows"] + 1, dtype=torch.int32, device="cuda")
+        ci = torch.empty((wl.num_q_heads, sz["nnz_per_head"]), dtype=torch.int32, device="cuda")
+        out = torch.empty((sz["total_tokens"], wl.num_q_heads, wl.head_dim), dtype=torch.bfloat16, device="cuda")
+        S.stem_score(prob, q, k, v, scores=scores, ws=ws)
+        S.stem_select(prob, scores, rp, ci, ws=ws)
+        for _ in range(args.warmup):
+            S.bsa_prefill(prob, q, k, v, rp, ci, out=out, ws=ws)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for a, b in evs:
+            a.record(stream)
+            S.bsa_prefill(prob, q, k, v, rp, ci, out=out, ws=ws)
+            b.record(stream)
+        torch.cuda.synchronize()
+        ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+        fl = selected_flops(prob, rp.cpu().numpy(), wl.block, wl.head_dim, wl.seqlens)
+        if dense_ms is None:
+            for _ in range(args.warmup):
+                S.bsa_dense_prefill(prob, q, k, v, out=out, ws=ws)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(args.steps):
+                S.bsa_dense_prefill(prob, q, k, v, out=out, ws=ws)
+            b.record(stream)
+            torch.cuda.synchronize()
+            dense_ms = a.elapsed_time(b) / args.steps
+        S.query_status(ws)
+        rows.append({"keep": keep, "selected_tflop": fl / 1e12, "bsa_ms": ms, "tflops": fl / (ms * 1e-3) / 1e12,
+                     "fraction_of_dense_time": ms / dense_ms})
+    x = np.array([r["selected_tflop"] for r in rows])
+    y = np.array([r["bsa_ms"] for r in rows])
+    slope, icpt = np.polyfit(x, y, 1)
+    r2 = 1.0 - float(np.sum((y - (slope * x + icpt)) ** 2) / np.sum((y - y.mean()) ** 2))
+    line = {"metric": "BSA latency vs density (linear fit of ms on selected TFLOP)", "workload": wl.name,
+            "dtype": "e4m3" if wl.dtype == "fp8_e4m3" else "bf16", "steps": args.steps, "warmup": args.warmup,
+            "dense_ms": dense_ms, "sweep": rows,
+            "fit": {"ms_per_tflop": float(slope), "intercept_ms": float(icpt), "r2": r2}}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -208,6 +262,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="density sweep (keep 1.0 .. 0.1) against the dense kernel")
     args = ap.parse_args()
     wl = W.ALL[args.workload]
     if args.keep is not None:
@@ -216,6 +271,12 @@ def main():
         wl = wl.with_(seqlens=(args.seqlen,), name=f"{wl.name}@{args.seqlen}")
     if args.impl == "reference":
         run_reference(args, wl)
+        return
+    if args.sweep:
+        if not torch.cuda.is_available():
+            raise SystemExit("bench.py needs a CUDA device (the path has no CPU fallback)")
+        S.lib()
+        run_sweep(args)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <map>
 #include <mutex>
@@ -351,6 +352,10 @@ stem_status_t check_qkv(const void* q, const void* k, const void* v, const stem_
 
 }  // namespace
 
+std::atomic<int> g_inject{0};
+int take_injection() { return g_inject.exchange(0); }
+void set_injection(int mode) { g_inject.store(mode); }
+
 stem_status_t set_last_error(stem_status_t s, const char* fmt, ...) {
   va_list ap;
   va_start(ap, fmt);
@@ -523,5 +528,11 @@ const char* stem_status_string(stem_status_t s) {
 }
 
 const char* stem_last_error(void) { return g_err; }
+
+stem_status_t stem_debug_inject(int mode) {
+  if (mode != 0 && mode != 1) return fail(STEM_ERR_INVALID, "unknown injection mode %d", mode);
+  set_injection(mode);
+  return STEM_OK;
+}
 
 }  // extern "C"

@@ -100,6 +100,7 @@ struct BsaParams {
   float out_scale;   // FP8: v_scale (l carries the P factor); BF16: 1
   float p_scale;     // the factor itself (1 for BF16)
   uint32_t* status;
+  int inject;        // 1: CTA 0 withholds its first K tile (failure-detection test)
   signed char order[STEM_MAX_SEQS];  // sequences by decreasing block count
 };
 
@@ -288,7 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
           for (int hh = 0; hh < C::HALVES; ++hh) rows[hh] = __shfl_sync(full, rowh[hh], q);
           const uint32_t ks = itk % C::KST, kph = (itk / C::KST) & 1;
           if (!warp_wait(bar_k_empty + 8 * ks, kph ^ 1, abort_flag, p.status)) { alive = false; break; }
-          if (lane == 0) {
+          const bool withhold = p.inject == 1 && blockIdx.x == 0 && itk == 0;
+          if (lane == 0 && !withhold) {
             mbar_arrive_expect_tx(bar_k_full + 8 * ks, C::KV_BYTES);
             for (int c = 0; c < C::DCH; ++c)
               for (int hh = 0; hh < C::HALVES; ++hh)
@@ -654,6 +656,7 @@ cudaError_t launch_bsa(const Batch& bt, const BsaArgs& a, bool fp8, bool paged, 
   prm.Hq = a.Hq;
   prm.Hkv = a.Hkv;
   prm.status = status;
+  prm.inject = take_injection();
   const float log2e = 1.4426950408889634f;
   prm.scale_log2 = a.sigma * (fp8 ? a.q_scale * a.k_scale : 1.0f) * log2e;
   // FP8: P <= 2^8 after the lazy max update; 448 / 256 keeps it inside e4m3's range.

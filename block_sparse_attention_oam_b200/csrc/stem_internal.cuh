@@ -410,4 +410,8 @@ struct BsaArgs {
 cudaError_t launch_bsa(const Batch& bt, const BsaArgs& a, bool fp8, bool paged, bool dense, uint32_t* status,
                        cudaStream_t st);
 
+// Pending failure-injection request (stem_debug_inject); consumed by the next BSA launch.
+int take_injection();
+void set_injection(int mode);
+
 }  // namespace stem

@@ -99,6 +99,7 @@ def lib() -> ctypes.CDLL:
         "stem_reset_status": ([_P, _P], ctypes.c_int),
         "stem_status_string": ([ctypes.c_int], ctypes.c_char_p),
         "stem_last_error": ([], ctypes.c_char_p),
+        "stem_debug_inject": ([ctypes.c_int], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -263,6 +264,12 @@ def stem_attention_noalloc(prob: Problem, q, k, v, paged: Optional[PagedKV] = No
     _check(lib().stem_attention_noalloc(prob.c, _ptr(q), _ptr(k), _ptr(v), _paged(paged), _ptr(out), _ptr(lse),
                                         _ptr(row_ptr), _ptr(col_idx), _ptr(status), _stream(stream)))
     return out
+
+
+def debug_inject(mode: int) -> None:
+    """Failure-detection test hook: mode 1 makes the next BSA launch stall one CTA
+    until its bounded wait reports STEM_ERR_TIMEOUT."""
+    _check(lib().stem_debug_inject(mode))
 
 
 def query_status(ws, stream=None) -> int:

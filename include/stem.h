@@ -209,6 +209,16 @@ STEM_API stem_status_t stem_query_status(void* ws, void* stream);
 /* Zero the workspace status word (enqueued on the stream). */
 STEM_API stem_status_t stem_reset_status(void* ws, void* stream);
 
+/*
+ * Failure-detection test hook (no counterpart in the pages).  mode 1 makes the next
+ * bsa_prefill / bsa_dense_prefill / stem_attention launch withhold one K tile in
+ * the first CTA, so that CTA's bounded pipeline wait runs out (after about 2 s):
+ * the kernel records STEM_ERR_TIMEOUT in the workspace status word, releases its
+ * tensor memory and exits, and the GPU context stays usable.  The launch that
+ * consumes the request clears it; mode 0 cancels a pending request.
+ */
+STEM_API stem_status_t stem_debug_inject(int mode);
+
 /* Static description of a status code. */
 STEM_API const char* stem_status_string(stem_status_t s);
 

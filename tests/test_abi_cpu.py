@@ -22,7 +22,7 @@ def test_library_exports_every_declared_function(L):
     names = S.header_functions()
     expect = {"stem_query_sizes", "stem_workspace_size", "stem_tpd_plan", "stem_score", "stem_select",
               "bsa_prefill", "bsa_dense_prefill", "stem_attention", "stem_query_status", "stem_reset_status",
-              "stem_status_string", "stem_last_error"}
+              "stem_status_string", "stem_last_error", "stem_attention_noalloc", "stem_debug_inject"}
     assert expect <= set(names), set(names)
     for n in names:
         assert hasattr(L, n), n
