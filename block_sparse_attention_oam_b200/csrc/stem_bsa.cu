@@ -7,23 +7,26 @@
 // being -inf, so the softmax stays exact; the inner path is the dense one.  The
 // same section notes native support for a paged KV cache.
 //
-// Design (one CTA per SM, persistent over (q-head, q-block) tiles, 10 warps):
-//   warp 0      TMA producer: the Q tile once per tile, then K_j and V_j of every listed
-//               block into separate rings (64-row boxes, 128-byte swizzle; a paged cache
-//               is read page by page through the block table).
-//   warp 1      MMA issuer (one thread): S = Q K_j^T into one of two TMEM S buffers, then
-//               O += P_j V_j with P read from TMEM (where the softmax wrote it over S_j)
-//               and V from shared memory.  S_{j+1} is issued before P_j is ready, so the
-//               tensor core overlaps the softmax.
-//   warps 2..9  softmax, two warpgroups: each query row is shared by two threads, one per
-//               warpgroup, each owning half of every KV block's columns.  The halves run
-//               independent online softmaxes (own running max, own sum, own O accumulator
-//               in TMEM) and are merged once per tile in the epilogue, so no per-block
-//               exchange between them is needed.  Log2 domain, packed fp32x2 arithmetic;
-//               the token-level causal mask only on the diagonal block (always the last
-//               list entry); lazy rescaling of O (only when a running max grows by more
-//               than 2^8), waiting for the previous P V product only then; O normalised
-//               by the sum of the rounded P weights the product used.
+// Design (one CTA per SM, persistent, 10 warps).  Work unit: one q-block row i of one
+// sequence for a PAIR of q-heads (2p, 2p+1).  Both tiles of a pair list the same number of
+// blocks (the budget k_i does not depend on the head), so they advance in lock-step in
+// two "slots" that share the tensor core (ping-pong): while the softmax of one slot works
+// on its scores, the tensor core runs the other slot's P V and next S.
+//   warp 0      TMA producer: per slot, the Q tile once per unit, then K_j and V_j of
+//               every listed block into per-slot rings (64-row boxes, 128-byte swizzle;
+//               a paged cache is read page by page through the block table).
+//   warp 1      MMA issuer (one thread): per slot, S = Q K_j^T into the slot's TMEM S/P
+//               columns, then O += P_j V_j with P read from TMEM (where the softmax wrote
+//               it over S_j) and V from shared memory.  Order per block j:
+//               PV_0(j), S_0(j+1), PV_1(j), S_1(j+1).
+//   warps 2..5  softmax of slot 0, warps 6..9 softmax of slot 1: one thread per query row
+//               (TMEM lane quadrant = warp % 4).  Online softmax in the log2 domain with
+//               packed fp32x2 arithmetic; the token-level causal mask only on the diagonal
+//               block (always the last list entry); O rescaled lazily (only when the
+//               running max grows by more than 2^8) — no wait is needed for that, since
+//               S_j is issued after P V_{j-1} and the tensor core runs in order; O
+//               normalised by the sum of the rounded P weights the product used; then the
+//               epilogue (O / l -> bf16, log-sum-exp).
 // Every wait is bounded (2 s); on expiry the CTA raises an abort flag, records
 // STEM_ERR_TIMEOUT in the status word, drains its tensor-core work, waits (bounded)
 // for its copies and releases its TMEM before exiting.
@@ -37,9 +40,8 @@ namespace stem {
 namespace {
 
 constexpr int kBM = 128;              // query rows per tile (tcgen05 M)
-constexpr int kSoftmaxWarps = 8;
-constexpr int kThreads = 64 + 32 * kSoftmaxWarps;
-constexpr uint32_t kTmemCols = 512;
+constexpr int kThreads = 64 + 256;    // producer, MMA, two softmax warpgroups
+constexpr uint32_t kTmemCols = 512;   // per slot: S/P at +0 (128 columns), O at +128 (D)
 constexpr uint32_t kSmemCap = 227 * 1024;
 
 template <int D, int BN, bool FP8>
@@ -56,23 +58,19 @@ struct Cfg {
   static constexpr int PV_KSTEPS = BN * ES / 32;  // MMAs along the KV block for O
   static constexpr int PV_KROWS = 32 / ES;        // KV rows consumed per PV MMA
   static constexpr int HALVES = BN / 64;          // 64-row TMA boxes per KV block
-  static constexpr int HALF = BN / 2;             // S columns per softmax thread
-  static constexpr int P_COLS = HALF * ES / 4;    // TMEM columns of one thread's P (packed)
-  static constexpr int O_HALF = D / 2;            // output columns stored per softmax thread
-  static constexpr int PV_HSTEPS = PV_KSTEPS / 2; // P V MMAs per half (one O accumulator each)
-  static constexpr int EXTRA = 512 + 3072;        // barriers, per-tile (m, l, lt) exchange
+  static constexpr int P_COLS = BN * ES / 4;      // TMEM columns of a row's P (packed)
+  static constexpr int EXTRA = 512;               // barriers and flags
   static constexpr int SLACK = 1024;              // alignment of the tiles to 1024 bytes
-  // K / V ring depths: as deep as shared memory allows, at most 4
-  static constexpr int ROOM = static_cast<int>(kSmemCap) - Q_BYTES - EXTRA - SLACK;
-  static constexpr int KST = ROOM / KV_BYTES >= 8 ? 4 : (ROOM / KV_BYTES >= 6 ? 3 : 2);
-  static constexpr int VST = ROOM / KV_BYTES >= 8 ? 4 : (ROOM / KV_BYTES >= 5 ? (ROOM / KV_BYTES) - KST : 2);
-  static_assert(KST + VST <= ROOM / KV_BYTES, "K/V rings do not fit");
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
-  static constexpr int OFF_XCH = OFF_BAR + 512;    // float [3 kind][2 wg][128]
-  static constexpr int SMEM = OFF_XCH + 3072 + SLACK;
+  // per-slot K and V ring depth: as deep as shared memory allows, at most 4
+  static constexpr int ROOM = static_cast<int>(kSmemCap) - 2 * Q_BYTES - EXTRA - SLACK;
+  static constexpr int NST0 = ROOM / (4 * KV_BYTES);
+  static constexpr int NST = NST0 > 4 ? 4 : (NST0 < 1 ? 1 : NST0);
+  static_assert(4 * NST * KV_BYTES <= ROOM, "K/V rings do not fit");
+  static constexpr int OFF_Q = 0;                               // [slot]
+  static constexpr int OFF_K = 2 * Q_BYTES;                     // [slot][stage]
+  static constexpr int OFF_V = OFF_K + 2 * NST * KV_BYTES;      // [slot][stage]
+  static constexpr int OFF_BAR = OFF_V + 2 * NST * KV_BYTES;
+  static constexpr int SMEM = OFF_BAR + EXTRA + SLACK;
   // force one CTA per SM (the TMEM allocation takes all 512 columns)
   static constexpr int SMEM_LAUNCH = SMEM < 120 * 1024 ? 120 * 1024 : SMEM;
   static_assert(SMEM <= static_cast<int>(kSmemCap), "shared memory budget exceeded");
@@ -94,7 +92,7 @@ struct BsaParams {
   void* out;
   float* lse;
   int Hq, Hkv;
-  int total_tiles;
+  int total_units;   // sum over sequences of N_b * ceil(Hq / 2)
   float scale_log2;  // sigma * q_scale * k_scale * log2(e)
   float p_bias;      // log2 of the factor P is scaled by before rounding (FP8: log2 1.75)
   float out_scale;   // FP8: v_scale (l carries the P factor); BF16: 1
@@ -104,31 +102,32 @@ struct BsaParams {
   signed char order[STEM_MAX_SEQS];  // sequences by decreasing block count
 };
 
-struct Tile {
-  int b, i, h;
+struct Unit {
+  int b, i, h0;      // sequence, q-block row, first q-head of the pair
+  bool two;          // the pair's second head exists
 };
 
-// Tile order: sequences by decreasing length; inside a sequence kv-head by kv-head, rows
-// from the last (longest list) to the first, the g q-heads of a row adjacent.  The CTAs
-// running at one time then share one kv-head's K/V, which fits in L2.
-__device__ __forceinline__ Tile decode_tile(const BsaParams& p, int t) {
-  Tile r{0, 0, 0};
-  const int G = p.Hq / p.Hkv;
+// Unit order: sequences by decreasing length; inside a sequence head pair by head pair,
+// rows from the last (longest list) to the first.  The CTAs running at one time then
+// share one pair's kv-head(s), whose K/V fit in L2.
+__device__ __forceinline__ Unit decode_unit(const BsaParams& p, int u) {
+  Unit r{0, 0, 0, false};
+  const int NP = (p.Hq + 1) / 2;
   int acc = 0;
   for (int q = 0; q < p.bt.num_seqs; ++q) {
     const int b = p.order[q];
     const int nb = p.bt.seq[b].nblk;
-    const int nt = nb * p.Hq;
-    if (t < acc + nt) {
-      const int local = t - acc;
-      const int kvh = local / (nb * G);
-      const int rem = local - kvh * nb * G;
+    const int nu = nb * NP;
+    if (u < acc + nu) {
+      const int local = u - acc;
+      const int pair = local / nb;
       r.b = b;
-      r.i = nb - 1 - rem / G;
-      r.h = kvh * G + rem % G;
+      r.i = nb - 1 - (local - pair * nb);
+      r.h0 = 2 * pair;
+      r.two = r.h0 + 1 < p.Hq;
       return r;
     }
-    acc += nt;
+    acc += nu;
   }
   return r;
 }
@@ -156,19 +155,18 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
-// Number of listed blocks of a tile and a pointer to its list (dense: implicit 0..i).
+// Number of listed blocks of a row (the same for every head) and a head's list
+// (dense: implicit 0..i).
 template <bool DENSE>
-__device__ __forceinline__ int tile_len(const BsaParams& p, const Tile& t, const int32_t** list) {
-  if (DENSE) {
-    *list = nullptr;
-    return t.i + 1;
-  }
-  const SeqInfo& s = p.bt.seq[t.b];
-  const int row = s.row0 + t.i;
-  const int beg = p.row_ptr[row];
-  const int n = p.row_ptr[row + 1] - beg;
-  *list = p.col_idx + static_cast<long long>(t.h) * p.bt.nnz_per_head + beg;
-  return (n >= 1 && n <= t.i + 1) ? n : 0;
+__device__ __forceinline__ int unit_len(const BsaParams& p, const Unit& un) {
+  if (DENSE) return un.i + 1;
+  const int row = p.bt.seq[un.b].row0 + un.i;
+  const int n = p.row_ptr[row + 1] - p.row_ptr[row];
+  return (n >= 1 && n <= un.i + 1) ? n : 0;
+}
+__device__ __forceinline__ const int32_t* head_list(const BsaParams& p, const Unit& un, int h) {
+  const int row = p.bt.seq[un.b].row0 + un.i;
+  return p.col_idx + static_cast<long long>(h) * p.bt.nnz_per_head + p.row_ptr[row];
 }
 
 template <int D, int BN, bool FP8, bool PAGED, bool DENSE>
@@ -182,36 +180,37 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
   const uint32_t sK = sbase + C::OFF_K;
   const uint32_t sV = sbase + C::OFF_V;
   unsigned char* bar_area = smem + C::OFF_BAR;
-  float* xch = reinterpret_cast<float*>(smem + C::OFF_XCH);
-  // barriers (8 bytes each)
+  // per-slot barriers (8 bytes each), slot s at b0 + 192 s
   const uint32_t b0 = sbase + C::OFF_BAR;
-  const uint32_t bar_q_full = b0 + 0, bar_q_empty = b0 + 8;
-  const uint32_t bar_k_full = b0 + 16, bar_k_empty = b0 + 48;   // [4]
-  const uint32_t bar_v_full = b0 + 80, bar_v_empty = b0 + 112;  // [4]
-  const uint32_t bar_s_full = b0 + 144;                         // [2]
-  const uint32_t bar_p_full = b0 + 160, bar_pv_done = b0 + 168;
-  const uint32_t bar_drain = b0 + 176, bar_x = b0 + 184;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_area + 256);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 264);
+  auto q_full = [&](int s) { return b0 + 192 * s + 0; };
+  auto q_empty = [&](int s) { return b0 + 192 * s + 8; };
+  auto k_full = [&](int s, int t) { return b0 + 192 * s + 16 + 8 * t; };
+  auto k_empty = [&](int s, int t) { return b0 + 192 * s + 48 + 8 * t; };
+  auto v_full = [&](int s, int t) { return b0 + 192 * s + 80 + 8 * t; };
+  auto v_empty = [&](int s, int t) { return b0 + 192 * s + 112 + 8 * t; };
+  auto s_full = [&](int s) { return b0 + 192 * s + 144; };
+  auto p_full = [&](int s) { return b0 + 192 * s + 152; };
+  auto o_done = [&](int s) { return b0 + 192 * s + 160; };
+  const uint32_t bar_drain = b0 + 384;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_area + 448);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 456);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (threadIdx.x == 0) {
-    mbar_init(bar_q_full, 1);
-    mbar_init(bar_q_empty, 1);
-    for (int s = 0; s < C::KST; ++s) {
-      mbar_init(bar_k_full + 8 * s, 1);
-      mbar_init(bar_k_empty + 8 * s, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(q_full(s), 1);
+      mbar_init(q_empty(s), 1);
+      for (int t = 0; t < C::NST; ++t) {
+        mbar_init(k_full(s, t), 1);
+        mbar_init(k_empty(s, t), 1);
+        mbar_init(v_full(s, t), 1);
+        mbar_init(v_empty(s, t), 1);
+      }
+      mbar_init(s_full(s), 1);
+      mbar_init(p_full(s), 4);
+      mbar_init(o_done(s), 1);
     }
-    for (int s = 0; s < C::VST; ++s) {
-      mbar_init(bar_v_full + 8 * s, 1);
-      mbar_init(bar_v_empty + 8 * s, 1);
-    }
-    mbar_init(bar_s_full, 1);
-    mbar_init(bar_s_full + 8, 1);
-    mbar_init(bar_p_full, kSoftmaxWarps);
-    mbar_init(bar_pv_done, 1);
     mbar_init(bar_drain, 1);
-    mbar_init(bar_x, kSoftmaxWarps);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -223,9 +222,6 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_S = tmem;          // two S buffers at columns 0 and 128 (P overwrites S)
-  const uint32_t tmem_O = tmem + 256;    // O of half 0 at 256, of half 1 at 256 + D
-
   const int G = p.Hq / p.Hkv;
   const unsigned full = 0xffffffffu;
 
@@ -236,160 +232,175 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
       tma_prefetch_map(&p.tk);
       tma_prefetch_map(&p.tv);
     }
-    uint32_t itk = 0, itv = 0, tq = 0;
+    uint32_t itk[2] = {0, 0}, itv[2] = {0, 0}, tq = 0;
     bool alive = true;
-    for (int t = blockIdx.x; t < p.total_tiles && alive; t += gridDim.x) {
-      const Tile tl = decode_tile(p, t);
-      const int32_t* list;
-      const int n = tile_len<DENSE>(p, tl, &list);
+    for (int u = blockIdx.x; u < p.total_units && alive; u += gridDim.x) {
+      const Unit un = decode_unit(p, u);
+      const int n = unit_len<DENSE>(p, un);
       if (n == 0) {
         if (lane == 0) atomicOr(p.status, kStatusBounds);
         continue;
       }
-      const SeqInfo& s = p.bt.seq[tl.b];
-      const int kvh = tl.h / G;
-      if (!warp_wait(bar_q_empty, (tq & 1) ^ 1, abort_flag, p.status)) { alive = false; break; }
-      if (lane == 0) {
-        mbar_arrive_expect_tx(bar_q_full, C::Q_BYTES);
-        for (int c = 0; c < C::DCH; ++c)
-          tma_load_3d(sQ + c * C::Q_CHUNK, &p.tq, bar_q_full, c * C::CH, tl.h, s.tok0 + tl.i * BN);
+      const int ns = un.two ? 2 : 1;
+      const SeqInfo& sq = p.bt.seq[un.b];
+      for (int s = 0; s < ns; ++s) {
+        if (!warp_wait(q_empty(s), (tq & 1) ^ 1, abort_flag, p.status)) { alive = false; break; }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(q_full(s), C::Q_BYTES);
+          for (int c = 0; c < C::DCH; ++c)
+            tma_load_3d(sQ + s * C::Q_BYTES + c * C::Q_CHUNK, &p.tq, q_full(s), c * C::CH, un.h0 + s,
+                        sq.tok0 + un.i * BN);
+        }
       }
+      if (!alive) break;
       ++tq;
-      const int npages = (s.len + STEM_PAGE_SIZE - 1) / STEM_PAGE_SIZE;
+      const int npages = (sq.len + STEM_PAGE_SIZE - 1) / STEM_PAGE_SIZE;
+      const int32_t* lists[2] = {DENSE ? nullptr : head_list(p, un, un.h0),
+                                 DENSE || !un.two ? nullptr : head_list(p, un, un.h0 + 1)};
       for (int j0 = 0; j0 < n && alive; j0 += 32) {
         const int jl = j0 + lane;
-        int myj = jl;
-        if (!DENSE) myj = jl < n ? __ldg(list + jl) : 0;
-        if (jl < n && (myj < 0 || myj > tl.i)) {
-          atomicOr(p.status, kStatusBounds);
-          myj = tl.i;
-        }
-        if (jl >= n) myj = 0;
-        // rows of this lane's block (one per 64-row box), resolved through the block table
-        int rowh[C::HALVES];
+        // rows of this lane's block for each slot (one per 64-row box)
+        int rowh[2][C::HALVES];
 #pragma unroll
-        for (int hh = 0; hh < C::HALVES; ++hh) {
-          if (PAGED) {
-            int pg = (myj * BN) / STEM_PAGE_SIZE + hh;
-            pg = pg < npages ? pg : npages - 1;
-            int slot = (jl < n) ? __ldg(p.block_table + static_cast<long long>(tl.b) * p.max_pages + pg) : 0;
-            if (slot < 0 || slot >= p.num_slots) {
-              atomicOr(p.status, kStatusBounds);
-              slot = 0;
+        for (int s = 0; s < 2; ++s) {
+          int myj = jl;
+          if (!DENSE) myj = (jl < n && s < ns) ? __ldg(lists[s] + jl) : 0;
+          if (jl < n && s < ns && (myj < 0 || myj > un.i)) {
+            atomicOr(p.status, kStatusBounds);
+            myj = un.i;
+          }
+          if (jl >= n || s >= ns) myj = 0;
+#pragma unroll
+          for (int hh = 0; hh < C::HALVES; ++hh) {
+            if (PAGED) {
+              int pg = (myj * BN) / STEM_PAGE_SIZE + hh;
+              pg = pg < npages ? pg : npages - 1;
+              int slot = (jl < n && s < ns) ? __ldg(p.block_table + static_cast<long long>(un.b) * p.max_pages + pg) : 0;
+              if (slot < 0 || slot >= p.num_slots) {
+                atomicOr(p.status, kStatusBounds);
+                slot = 0;
+              }
+              rowh[s][hh] = slot * STEM_PAGE_SIZE;
+            } else {
+              rowh[s][hh] = sq.tok0 + myj * BN + hh * 64;
             }
-            rowh[hh] = slot * STEM_PAGE_SIZE;
-          } else {
-            rowh[hh] = s.tok0 + myj * BN + hh * 64;
           }
         }
         const int cnt = min(32, n - j0);
-        for (int q = 0; q < cnt; ++q) {
-          int rows[C::HALVES];
+        for (int q = 0; q < cnt && alive; ++q) {
+          int rows[2][C::HALVES];
 #pragma unroll
-          for (int hh = 0; hh < C::HALVES; ++hh) rows[hh] = __shfl_sync(full, rowh[hh], q);
-          const uint32_t ks = itk % C::KST, kph = (itk / C::KST) & 1;
-          if (!warp_wait(bar_k_empty + 8 * ks, kph ^ 1, abort_flag, p.status)) { alive = false; break; }
-          const bool withhold = p.inject == 1 && blockIdx.x == 0 && itk == 0;
-          if (lane == 0 && !withhold) {
-            mbar_arrive_expect_tx(bar_k_full + 8 * ks, C::KV_BYTES);
-            for (int c = 0; c < C::DCH; ++c)
-              for (int hh = 0; hh < C::HALVES; ++hh)
-                tma_load_3d(sK + ks * C::KV_BYTES + c * C::KV_CHUNK + hh * 64 * 128, &p.tk, bar_k_full + 8 * ks,
-                            c * C::CH, kvh, rows[hh]);
+          for (int s = 0; s < 2; ++s)
+#pragma unroll
+            for (int hh = 0; hh < C::HALVES; ++hh) rows[s][hh] = __shfl_sync(full, rowh[s][hh], q);
+          for (int s = 0; s < ns; ++s) {
+            const int kvh = (un.h0 + s) / G;
+            const uint32_t t = itk[s] % C::NST, ph = (itk[s] / C::NST) & 1;
+            if (!warp_wait(k_empty(s, t), ph ^ 1, abort_flag, p.status)) { alive = false; break; }
+            const bool withhold = p.inject == 1 && blockIdx.x == 0 && s == 0 && itk[0] == 0;
+            if (lane == 0 && !withhold) {
+              mbar_arrive_expect_tx(k_full(s, t), C::KV_BYTES);
+              for (int c = 0; c < C::DCH; ++c)
+                for (int hh = 0; hh < C::HALVES; ++hh)
+                  tma_load_3d(sK + (s * C::NST + t) * C::KV_BYTES + c * C::KV_CHUNK + hh * 64 * 128, &p.tk,
+                              k_full(s, t), c * C::CH, kvh, rows[s][hh]);
+            }
+            ++itk[s];
           }
-          ++itk;
-          const uint32_t vs = itv % C::VST, vph = (itv / C::VST) & 1;
-          if (!warp_wait(bar_v_empty + 8 * vs, vph ^ 1, abort_flag, p.status)) { alive = false; break; }
-          if (lane == 0) {
-            mbar_arrive_expect_tx(bar_v_full + 8 * vs, C::KV_BYTES);
-            for (int c = 0; c < C::DCH; ++c)
-              for (int hh = 0; hh < C::HALVES; ++hh)
-                tma_load_3d(sV + vs * C::KV_BYTES + c * C::KV_CHUNK + hh * 64 * 128, &p.tv, bar_v_full + 8 * vs,
-                            c * C::CH, kvh, rows[hh]);
+          for (int s = 0; s < ns && alive; ++s) {
+            const int kvh = (un.h0 + s) / G;
+            const uint32_t t = itv[s] % C::NST, ph = (itv[s] / C::NST) & 1;
+            if (!warp_wait(v_empty(s, t), ph ^ 1, abort_flag, p.status)) { alive = false; break; }
+            if (lane == 0) {
+              mbar_arrive_expect_tx(v_full(s, t), C::KV_BYTES);
+              for (int c = 0; c < C::DCH; ++c)
+                for (int hh = 0; hh < C::HALVES; ++hh)
+                  tma_load_3d(sV + (s * C::NST + t) * C::KV_BYTES + c * C::KV_CHUNK + hh * 64 * 128, &p.tv,
+                              v_full(s, t), c * C::CH, kvh, rows[s][hh]);
+            }
+            ++itv[s];
           }
-          ++itv;
         }
       }
     }
     if (!alive) {
       // let the copies already issued land before the CTA can exit
-      for (uint32_t q = (itk > C::KST ? itk - C::KST : 0); q < itk; ++q)
-        for (int spin = 0; spin < 1000000 && !mbar_try_wait(bar_k_full + 8 * (q % C::KST), (q / C::KST) & 1); ++spin) {}
-      for (uint32_t q = (itv > C::VST ? itv - C::VST : 0); q < itv; ++q)
-        for (int spin = 0; spin < 1000000 && !mbar_try_wait(bar_v_full + 8 * (q % C::VST), (q / C::VST) & 1); ++spin) {}
+      for (int s = 0; s < 2; ++s) {
+        for (uint32_t q = (itk[s] > C::NST ? itk[s] - C::NST : 0); q < itk[s]; ++q)
+          for (int spin = 0; spin < 1000000 && !mbar_try_wait(k_full(s, q % C::NST), (q / C::NST) & 1); ++spin) {}
+        for (uint32_t q = (itv[s] > C::NST ? itv[s] - C::NST : 0); q < itv[s]; ++q)
+          for (int spin = 0; spin < 1000000 && !mbar_try_wait(v_full(s, q % C::NST), (q / C::NST) & 1); ++spin) {}
+      }
       if (tq > 0)
-        for (int spin = 0; spin < 1000000 && !mbar_try_wait(bar_q_full, (tq - 1) & 1); ++spin) {}
+        for (int s = 0; s < 2; ++s)
+          for (int spin = 0; spin < 1000000 && !mbar_try_wait(q_full(s), (tq - 1) & 1); ++spin) {}
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    uint32_t itk = 0, itv = 0, is = 0, ip = 0, tq = 0;
+    uint32_t itk[2] = {0, 0}, itv[2] = {0, 0}, gb[2] = {0, 0}, tq = 0;
     bool alive = true;
-    auto issue_s = [&](void) -> bool {
-      const uint32_t sb = is % 2;
-      const uint32_t ks = itk % C::KST, kph = (itk / C::KST) & 1;
-      if (!warp_wait(bar_k_full + 8 * ks, kph, abort_flag, p.status)) return false;
+    // S = Q K^T of the slot's next block into its S/P columns
+    auto issue_s = [&](int s, bool last) -> bool {
+      const uint32_t t = itk[s] % C::NST, ph = (itk[s] / C::NST) & 1;
+      if (!warp_wait(k_full(s, t), ph, abort_flag, p.status)) return false;
       tc_fence_after();
       if (lane == 0) {
+        const uint32_t d_tmem = tmem + 256 * s;
 #pragma unroll
         for (int k = 0; k < C::S_KSTEPS; ++k) {
           const int c = k / 4, w = k % 4;
-          const uint64_t ad = smem_desc_sw128(sQ + c * C::Q_CHUNK + w * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(sK + ks * C::KV_BYTES + c * C::KV_CHUNK + w * 32, 16, 1024);
+          const uint64_t ad = smem_desc_sw128(sQ + s * C::Q_BYTES + c * C::Q_CHUNK + w * 32, 16, 1024);
+          const uint64_t bd =
+              smem_desc_sw128(sK + (s * C::NST + t) * C::KV_BYTES + c * C::KV_CHUNK + w * 32, 16, 1024);
           if (FP8)
-            mma_fp8(tmem_S + sb * 128, ad, bd, C::IDESC_S, k > 0);
+            mma_fp8(d_tmem, ad, bd, C::IDESC_S, k > 0);
           else
-            mma_bf16(tmem_S + sb * 128, ad, bd, C::IDESC_S, k > 0);
+            mma_bf16(d_tmem, ad, bd, C::IDESC_S, k > 0);
         }
-        mma_commit(bar_s_full + 8 * sb);
-        mma_commit(bar_k_empty + 8 * ks);
+        mma_commit(s_full(s));
+        mma_commit(k_empty(s, t));
+        if (last) mma_commit(q_empty(s));  // every S of this unit issued: Q may be replaced
       }
       __syncwarp();
-      ++is;
-      ++itk;
+      ++itk[s];
       return true;
     };
-    for (int t = blockIdx.x; t < p.total_tiles && alive; t += gridDim.x) {
-      const Tile tl = decode_tile(p, t);
-      const int32_t* list;
-      const int n = tile_len<DENSE>(p, tl, &list);
+    for (int u = blockIdx.x; u < p.total_units && alive; u += gridDim.x) {
+      const Unit un = decode_unit(p, u);
+      const int n = unit_len<DENSE>(p, un);
       if (n == 0) continue;
-      if (!warp_wait(bar_q_full, tq & 1, abort_flag, p.status)) { alive = false; break; }
+      const int ns = un.two ? 2 : 1;
+      for (int s = 0; s < ns && alive; ++s) {
+        if (!warp_wait(q_full(s), tq & 1, abort_flag, p.status)) { alive = false; break; }
+        if (!issue_s(s, n == 1)) { alive = false; break; }
+      }
       ++tq;
-      if (!issue_s()) { alive = false; break; }
-      for (int jj = 0; jj < n; ++jj) {
-        if (jj + 1 < n) {
-          if (!issue_s()) { alive = false; break; }
-        }
-        if (jj + 1 == n) {
-          if (lane == 0) mma_commit(bar_q_empty);  // all S MMAs of the tile issued
-          __syncwarp();
-        }
-        const uint32_t pb = ip % 2;
-        if (!warp_wait(bar_p_full, ip & 1, abort_flag, p.status)) { alive = false; break; }
-        ++ip;
-        const uint32_t vs = itv % C::VST, vph = (itv / C::VST) & 1;
-        if (!warp_wait(bar_v_full + 8 * vs, vph, abort_flag, p.status)) { alive = false; break; }
-        tc_fence_after();
-        if (lane == 0) {
+      for (int jj = 0; jj < n && alive; ++jj) {
+        for (int s = 0; s < ns; ++s) {
+          if (!warp_wait(p_full(s), gb[s] & 1, abort_flag, p.status)) { alive = false; break; }
+          ++gb[s];
+          const uint32_t t = itv[s] % C::NST, ph = (itv[s] / C::NST) & 1;
+          if (!warp_wait(v_full(s, t), ph, abort_flag, p.status)) { alive = false; break; }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t d_tmem = tmem + 256 * s + 128;
 #pragma unroll
-          for (int k = 0; k < C::PV_KSTEPS; ++k) {
-            // half hf of the block's keys: its P (in that half's S columns) into its own O
-            const int hf = k / C::PV_HSTEPS, kk = k % C::PV_HSTEPS;
-            const uint64_t bd =
-                smem_desc_sw128(sV + vs * C::KV_BYTES + k * C::PV_KROWS * 128, C::KV_CHUNK, 1024);
-            const uint32_t a_tmem = tmem_S + pb * 128 + hf * C::HALF + kk * 8;
-            const uint32_t d_tmem = tmem_O + hf * D;
-            const uint32_t acc = (jj > 0 || kk > 0) ? 1u : 0u;
-            if (FP8)
-              mma_fp8_ts(d_tmem, a_tmem, bd, C::IDESC_PV, acc);
-            else
-              mma_bf16_ts(d_tmem, a_tmem, bd, C::IDESC_PV, acc);
+            for (int k = 0; k < C::PV_KSTEPS; ++k) {
+              const uint64_t bd =
+                  smem_desc_sw128(sV + (s * C::NST + t) * C::KV_BYTES + k * C::PV_KROWS * 128, C::KV_CHUNK, 1024);
+              const uint32_t acc = (jj > 0 || k > 0) ? 1u : 0u;
+              if (FP8)
+                mma_fp8_ts(d_tmem, tmem + 256 * s + k * 8, bd, C::IDESC_PV, acc);
+              else
+                mma_bf16_ts(d_tmem, tmem + 256 * s + k * 8, bd, C::IDESC_PV, acc);
+            }
+            mma_commit(v_empty(s, t));
+            if (jj + 1 == n) mma_commit(o_done(s));
           }
-          mma_commit(bar_v_empty + 8 * vs);
-          mma_commit(bar_pv_done);
+          __syncwarp();
+          ++itv[s];
+          if (jj + 1 < n && !issue_s(s, jj + 2 == n)) { alive = false; break; }
         }
-        __syncwarp();
-        ++itv;
       }
     }
     // drain: every tcgen05.mma issued by this thread has completed
@@ -398,42 +409,40 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
     for (int spin = 0; spin < 4000000 && !mbar_try_wait(bar_drain, 0); ++spin) {}
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    const int wg = (warp - 2) / 4;                   // which half of the KV block's columns
+    const int slot = (warp - 2) / 4;                 // which tile of the pair
     const int quad = warp % 4;                       // TMEM lane quadrant of this warp
     const int r = quad * 32 + lane;                  // query row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t my_O = tmem_O + wg * D + lane_off;
+    const uint32_t my_S = tmem + 256 * slot + lane_off;
+    const uint32_t my_O = tmem + 256 * slot + 128 + lane_off;
     const float sl2 = p.scale_log2;
-    uint32_t gb = 0, ix = 0;                         // blocks processed by this CTA; exchanges
+    uint32_t gb = 0, ot = 0;                         // blocks and units processed by this slot
     bool alive = true;
-    for (int t = blockIdx.x; t < p.total_tiles && alive; t += gridDim.x) {
-      const Tile tl = decode_tile(p, t);
-      const int32_t* list;
-      const int n = tile_len<DENSE>(p, tl, &list);
-      if (n == 0) continue;
-      // per half: running max, sum of the rounded P the product uses (normalises O) and,
-      // for FP8, the sum of the unrounded P (log-sum-exp)
+    for (int u = blockIdx.x; u < p.total_units && alive; u += gridDim.x) {
+      const Unit un = decode_unit(p, u);
+      const int n = unit_len<DENSE>(p, un);
+      if (n == 0 || (slot == 1 && !un.two)) continue;
+      const int h = un.h0 + slot;
+      // running max; sums of the rounded P the product uses (normalise O) and, for FP8,
+      // of the unrounded P (log-sum-exp)
       float m_run = -INFINITY;
       float2 l2 = make_float2(0.f, 0.f), lt2 = make_float2(0.f, 0.f);
       for (int jj = 0; jj < n; ++jj, ++gb) {
-        const uint32_t sb = gb % 2, sph = (gb / 2) & 1;
-        if (!warp_wait(bar_s_full + 8 * sb, sph, abort_flag, p.status)) { alive = false; break; }
+        if (!warp_wait(s_full(slot), gb & 1, abort_flag, p.status)) { alive = false; break; }
         tc_fence_after();
-        const uint32_t my_S = tmem_S + sb * 128 + wg * C::HALF + lane_off;
-        uint32_t sr[C::HALF];
+        uint32_t sr[BN];
 #pragma unroll
-        for (int c = 0; c < C::HALF / 32; ++c) tmem_ld32(my_S + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+        for (int c = 0; c < BN / 32; ++c) tmem_ld32(my_S + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
         tmem_wait_ld();
-        const bool diag = (jj == n - 1);
-        if (diag) {
+        if (jj == n - 1) {
 #pragma unroll
-          for (int c = 0; c < C::HALF; ++c)
-            if (wg * C::HALF + c > r) sr[c] = __float_as_uint(-INFINITY);
+          for (int c = 0; c < BN; ++c)
+            if (c > r) sr[c] = __float_as_uint(-INFINITY);
         }
         // row maximum with four independent chains
         float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < C::HALF; c += 8)
+        for (int c = 0; c < BN; c += 8)
 #pragma unroll
           for (int q = 0; q < 4; ++q) mq[q] = max3f(mq[q], __uint_as_float(sr[c + 2 * q]), __uint_as_float(sr[c + 2 * q + 1]));
         const float mx = fmaxf(max3f(mq[0], mq[1], mq[2]), mq[3]);
@@ -441,133 +450,108 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
         const bool resc = m_new > m_run + 8.0f;
         const float m_use = resc ? m_new : m_run;
         const float alpha = resc ? ex2_approx(m_run - m_use) : 1.0f;
-        const float2 sc2 = make_float2(sl2, sl2);
-        // a half that has seen only masked keys so far (m = -inf) gets P = 0, not NaN
         const float m_sub = m_use == -INFINITY ? 0.f : m_use;
+        const float2 sc2 = make_float2(sl2, sl2);
         const float2 bias2 = make_float2(p.p_bias - m_sub, p.p_bias - m_sub);
-        // sums with four independent chains
         float2 sq[4], tq4[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           sq[q] = make_float2(0.f, 0.f);
           tq4[q] = make_float2(0.f, 0.f);
         }
-        uint32_t pk[C::P_COLS];
-        if (!FP8) {
+        // P is packed in place over the first P_COLS registers of sr (each pair or quad of
+        // scores is read before its packed word is written)
+        auto exps = [&](auto want_lse) {
+          if constexpr (!FP8) {
 #pragma unroll
-          for (int u = 0; u < C::HALF / 2; ++u) {
-            const float2 y = fma2(make_float2(__uint_as_float(sr[2 * u]), __uint_as_float(sr[2 * u + 1])), sc2, bias2);
-            const uint32_t w = pack_bf16x2(ex2_approx(y.x), ex2_approx(y.y));
-            pk[u] = w;
-            sq[u % 4] = add2(sq[u % 4], make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
-          }
-        } else {
-          // e4m3 P; its rounded values are summed as f16 pairs (exact enough: two e4m3
-          // codes per f16 add) and the unrounded values only when the LSE is requested
-          auto fp8_block = [&](auto want_lse) {
+            for (int u2 = 0; u2 < BN / 2; ++u2) {
+              const float2 y = fma2(make_float2(__uint_as_float(sr[2 * u2]), __uint_as_float(sr[2 * u2 + 1])), sc2, bias2);
+              const uint32_t w = pack_bf16x2(ex2_approx(y.x), ex2_approx(y.y));
+              sr[u2] = w;
+              sq[u2 % 4] = add2(sq[u2 % 4], make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
+            }
+          } else {
 #pragma unroll
-            for (int u = 0; u < C::HALF / 4; ++u) {
-              const float2 y0 = fma2(make_float2(__uint_as_float(sr[4 * u]), __uint_as_float(sr[4 * u + 1])), sc2, bias2);
-              const float2 y1 = fma2(make_float2(__uint_as_float(sr[4 * u + 2]), __uint_as_float(sr[4 * u + 3])), sc2, bias2);
+            for (int u4 = 0; u4 < BN / 4; ++u4) {
+              const float2 y0 = fma2(make_float2(__uint_as_float(sr[4 * u4]), __uint_as_float(sr[4 * u4 + 1])), sc2, bias2);
+              const float2 y1 = fma2(make_float2(__uint_as_float(sr[4 * u4 + 2]), __uint_as_float(sr[4 * u4 + 3])), sc2, bias2);
               const float2 e0 = make_float2(ex2_approx(y0.x), ex2_approx(y0.y));
               const float2 e1 = make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
-              const uint32_t lo = pack_e4m3x2(e0.x, e0.y);
-              const uint32_t hi = pack_e4m3x2(e1.x, e1.y);
-              pk[u] = __byte_perm(lo, hi, 0x5410);
-              sq[u % 4] = add2(sq[u % 4], e4m3x4_pairsum(pk[u]));
-              if constexpr (decltype(want_lse)::value) tq4[u % 4] = add2(tq4[u % 4], add2(e0, e1));
+              const uint32_t w = __byte_perm(pack_e4m3x2(e0.x, e0.y), pack_e4m3x2(e1.x, e1.y), 0x5410);
+              sr[u4] = w;
+              sq[u4 % 4] = add2(sq[u4 % 4], e4m3x4_pairsum(w));
+              if constexpr (decltype(want_lse)::value) tq4[u4 % 4] = add2(tq4[u4 % 4], add2(e0, e1));
             }
-          };
-          if (p.lse != nullptr)
-            fp8_block(std::true_type{});
-          else
-            fp8_block(std::false_type{});
-        }
+          }
+        };
+        if (FP8 && p.lse != nullptr)
+          exps(std::true_type{});
+        else
+          exps(std::false_type{});
         const float2 sum2 = add2(add2(sq[0], sq[1]), add2(sq[2], sq[3]));
         const float2 sumt2 = add2(add2(tq4[0], tq4[1]), add2(tq4[2], tq4[3]));
-        // P overwrites the first columns of this half's S, packed along columns
-        static_assert(C::P_COLS == 32 || C::P_COLS == 16, "P columns per half");
-        if constexpr (C::P_COLS == 32)
-          tmem_st32(my_S, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-        else
-          tmem_st16(my_S, &pk[0]);
+        static_assert(C::P_COLS % 32 == 0, "P columns");
+#pragma unroll
+        for (int c = 0; c < C::P_COLS / 32; ++c) tmem_st32(my_S + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
         const float2 a2 = make_float2(alpha, alpha);
         l2 = fma2(l2, a2, sum2);
         if (FP8) lt2 = fma2(lt2, a2, sumt2);
         if (jj > 0 && __any_sync(full, resc)) {
-          // O of this half holds the sum up to the previous block once its P V product is
-          // done (the barrier cannot be two phases ahead: the next product needs this warp)
-          if (!warp_wait(bar_pv_done, (gb - 1) & 1, abort_flag, p.status)) { alive = false; break; }
-          tc_fence_after();
+          // O holds the sum up to the previous block: S_j was issued after P V_{j-1},
+          // the tensor core runs in order, and S_j is complete
 #pragma unroll
-          for (int c = 0; c < D / 16; ++c) {
-            uint32_t o[16];
-            tmem_ld16(my_O + c * 16, o);
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(my_O + c * 32, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; e += 2) {
+            for (int e = 0; e < 32; e += 2) {
               const float2 v = mul2(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2);
               o[e] = __float_as_uint(v.x);
               o[e + 1] = __float_as_uint(v.y);
             }
-            tmem_st16(my_O + c * 16, o);
+            tmem_st32(my_O + c * 32, o);
           }
         }
         tmem_wait_st();
         m_run = m_use;
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_p_full);
+        if (lane == 0) mbar_arrive(p_full(slot));
       }
       if (!alive) break;
-      // epilogue: wait for the last P V product, merge the two halves, normalise, store
-      if (!warp_wait(bar_pv_done, (gb - 1) & 1, abort_flag, p.status)) { alive = false; break; }
+      // epilogue: wait for the unit's last P V product, normalise, store
+      if (!warp_wait(o_done(slot), ot & 1, abort_flag, p.status)) { alive = false; break; }
+      ++ot;
       tc_fence_after();
-      float* mine = xch + wg * 128 + r;
-      mine[0] = m_run;
-      mine[256] = l2.x + l2.y;
-      mine[512] = lt2.x + lt2.y;
-      __syncwarp();
-      if (lane == 0) {
-        __threadfence_block();
-        mbar_arrive(bar_x);
-      }
-      if (!warp_wait(bar_x, ix & 1, abort_flag, p.status)) { alive = false; break; }
-      ++ix;
-      const float m0 = xch[r], m1 = xch[128 + r];
-      const float l0 = xch[256 + r], l1 = xch[384 + r];
-      const float t0 = xch[512 + r], t1 = xch[640 + r];
-      const float mf = fmaxf(m0, m1);
-      const float f0 = ex2_approx(m0 - mf), f1 = ex2_approx(m1 - mf);
-      const float l = l0 * f0 + l1 * f1;
+      const float l = l2.x + l2.y;
       const float inv = p.out_scale / l;
-      const float g0 = f0 * inv, g1 = f1 * inv;
-      const SeqInfo& s = p.bt.seq[tl.b];
-      const int rows_valid = min(BN, s.len - tl.i * BN);
-      const long long tok = static_cast<long long>(s.tok0) + tl.i * BN + r;
-      unsigned char* orow = static_cast<unsigned char*>(p.out) + ((tok * p.Hq + tl.h) * D + wg * C::O_HALF) * 2;
-      const float2 gg0 = make_float2(g0, g0), gg1 = make_float2(g1, g1);
+      const SeqInfo& sq = p.bt.seq[un.b];
+      const int rows_valid = min(BN, sq.len - un.i * BN);
+      const long long tok = static_cast<long long>(sq.tok0) + un.i * BN + r;
+      unsigned char* orow = static_cast<unsigned char*>(p.out) + (tok * p.Hq + h) * D * 2;
+      const float2 ii = make_float2(inv, inv);
 #pragma unroll
-      for (int c = 0; c < C::O_HALF / 16; ++c) {
-        uint32_t oa[16], ob[16];
-        tmem_ld16(tmem_O + wg * C::O_HALF + lane_off + c * 16, oa);
-        tmem_ld16(tmem_O + D + wg * C::O_HALF + lane_off + c * 16, ob);
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(my_O + c * 32, o);
         tmem_wait_ld();
         if (r < rows_valid) {
-          uint32_t w[8];
 #pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            const float2 v = fma2(make_float2(__uint_as_float(oa[e]), __uint_as_float(oa[e + 1])), gg0,
-                                  mul2(make_float2(__uint_as_float(ob[e]), __uint_as_float(ob[e + 1])), gg1));
-            w[e / 2] = pack_bf16x2(v.x, v.y);
+          for (int q = 0; q < 4; ++q) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 v = mul2(make_float2(__uint_as_float(o[8 * q + 2 * e]), __uint_as_float(o[8 * q + 2 * e + 1])), ii);
+              w[e] = pack_bf16x2(v.x, v.y);
+            }
+            *reinterpret_cast<uint4*>(orow + (c * 32 + 8 * q) * 2) = make_uint4(w[0], w[1], w[2], w[3]);
           }
-          *reinterpret_cast<uint4*>(orow + c * 32) = make_uint4(w[0], w[1], w[2], w[3]);
-          *reinterpret_cast<uint4*>(orow + c * 32 + 16) = make_uint4(w[4], w[5], w[6], w[7]);
         }
       }
-      if (p.lse != nullptr && wg == 0 && r < rows_valid) {
-        const float lt = FP8 ? (t0 * f0 + t1 * f1) / p.p_scale : l;
-        p.lse[static_cast<long long>(tl.h) * p.bt.total_tokens + tok] = (mf + __log2f(lt)) * 0.69314718055994531f;
+      if (p.lse != nullptr && r < rows_valid) {
+        const float lt = FP8 ? (lt2.x + lt2.y) / p.p_scale : l;
+        p.lse[static_cast<long long>(h) * p.bt.total_tokens + tok] = (m_run + __log2f(lt)) * 0.69314718055994531f;
       }
       tc_fence_before();
     }
@@ -621,7 +605,7 @@ cudaError_t run(const BsaParams& prm, cudaStream_t st) {
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = prm.total_tiles < sms ? prm.total_tiles : sms;
+  const int grid = prm.total_units < sms ? prm.total_units : sms;
   if (grid <= 0) return cudaSuccess;
   kern<<<grid, kThreads, C::SMEM_LAUNCH, st>>>(prm);
   return cudaGetLastError();
@@ -664,9 +648,9 @@ cudaError_t launch_bsa(const Batch& bt, const BsaArgs& a, bool fp8, bool paged, 
   prm.p_bias = fp8 ? 0.80735492205760410f : 0.0f;  // log2(1.75)
   // l is accumulated from the scaled, rounded P, so the V scale is all that remains
   prm.out_scale = fp8 ? a.v_scale : 1.0f;
-  long long tiles = 0;
-  for (int b = 0; b < bt.num_seqs; ++b) tiles += static_cast<long long>(bt.seq[b].nblk) * a.Hq;
-  prm.total_tiles = static_cast<int>(tiles);
+  long long units = 0;
+  for (int b = 0; b < bt.num_seqs; ++b) units += static_cast<long long>(bt.seq[b].nblk) * ((a.Hq + 1) / 2);
+  prm.total_units = static_cast<int>(units);
   // sequences by decreasing block count (longest rows first)
   int ord[STEM_MAX_SEQS];
   for (int b = 0; b < bt.num_seqs; ++b) ord[b] = b;
