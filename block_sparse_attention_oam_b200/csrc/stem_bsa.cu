@@ -337,14 +337,15 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    uint32_t itk[2] = {0, 0}, itv[2] = {0, 0}, gb[2] = {0, 0}, tq = 0;
-    bool alive = true;
-    // S = Q K^T of the slot's next block into its S/P columns
-    auto issue_s = [&](int s, bool last) -> bool {
-      const uint32_t t = itk[s] % C::NST, ph = (itk[s] / C::NST) & 1;
-      if (!warp_wait(k_full(s, t), ph, abort_flag, p.status)) return false;
-      tc_fence_after();
-      if (lane == 0) {
+    // One thread does all of it: its waits and commits then cost no warp-wide votes.
+    if (lane == 0) {
+      uint32_t itk[2] = {0, 0}, itv[2] = {0, 0}, gb[2] = {0, 0}, tq = 0;
+      bool alive = true;
+      // S = Q K^T of the slot's next block into its S/P columns
+      auto issue_s = [&](int s, bool last) -> bool {
+        const uint32_t t = itk[s] % C::NST, ph = (itk[s] / C::NST) & 1;
+        if (!mbar_wait(k_full(s, t), ph, abort_flag, p.status)) return false;
+        tc_fence_after();
         const uint32_t d_tmem = tmem + 256 * s;
 #pragma unroll
         for (int k = 0; k < C::S_KSTEPS; ++k) {
@@ -360,29 +361,26 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
         mma_commit(s_full(s));
         mma_commit(k_empty(s, t));
         if (last) mma_commit(q_empty(s));  // every S of this unit issued: Q may be replaced
-      }
-      __syncwarp();
-      ++itk[s];
-      return true;
-    };
-    for (int u = blockIdx.x; u < p.total_units && alive; u += gridDim.x) {
-      const Unit un = decode_unit(p, u);
-      const int n = unit_len<DENSE>(p, un);
-      if (n == 0) continue;
-      const int ns = un.two ? 2 : 1;
-      for (int s = 0; s < ns && alive; ++s) {
-        if (!warp_wait(q_full(s), tq & 1, abort_flag, p.status)) { alive = false; break; }
-        if (!issue_s(s, n == 1)) { alive = false; break; }
-      }
-      ++tq;
-      for (int jj = 0; jj < n && alive; ++jj) {
-        for (int s = 0; s < ns; ++s) {
-          if (!warp_wait(p_full(s), gb[s] & 1, abort_flag, p.status)) { alive = false; break; }
-          ++gb[s];
-          const uint32_t t = itv[s] % C::NST, ph = (itv[s] / C::NST) & 1;
-          if (!warp_wait(v_full(s, t), ph, abort_flag, p.status)) { alive = false; break; }
-          tc_fence_after();
-          if (lane == 0) {
+        ++itk[s];
+        return true;
+      };
+      for (int u = blockIdx.x; u < p.total_units && alive; u += gridDim.x) {
+        const Unit un = decode_unit(p, u);
+        const int n = unit_len<DENSE>(p, un);
+        if (n == 0) continue;
+        const int ns = un.two ? 2 : 1;
+        for (int s = 0; s < ns && alive; ++s) {
+          if (!mbar_wait(q_full(s), tq & 1, abort_flag, p.status)) { alive = false; break; }
+          if (!issue_s(s, n == 1)) { alive = false; break; }
+        }
+        ++tq;
+        for (int jj = 0; jj < n && alive; ++jj) {
+          for (int s = 0; s < ns; ++s) {
+            const uint32_t t = itv[s] % C::NST, ph = (itv[s] / C::NST) & 1;
+            if (!mbar_wait(v_full(s, t), ph, abort_flag, p.status)) { alive = false; break; }
+            if (!mbar_wait(p_full(s), gb[s] & 1, abort_flag, p.status)) { alive = false; break; }
+            ++gb[s];
+            tc_fence_after();
             const uint32_t d_tmem = tmem + 256 * s + 128;
 #pragma unroll
             for (int k = 0; k < C::PV_KSTEPS; ++k) {
@@ -396,17 +394,16 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
             }
             mma_commit(v_empty(s, t));
             if (jj + 1 == n) mma_commit(o_done(s));
+            ++itv[s];
+            if (jj + 1 < n && !issue_s(s, jj + 2 == n)) { alive = false; break; }
           }
-          __syncwarp();
-          ++itv[s];
-          if (jj + 1 < n && !issue_s(s, jj + 2 == n)) { alive = false; break; }
         }
       }
+      // drain: every tcgen05.mma issued by this thread has completed
+      mma_commit(bar_drain);
+      for (int spin = 0; spin < 4000000 && !mbar_try_wait(bar_drain, 0); ++spin) {}
     }
-    // drain: every tcgen05.mma issued by this thread has completed
-    if (lane == 0) mma_commit(bar_drain);
     __syncwarp();
-    for (int spin = 0; spin < 4000000 && !mbar_try_wait(bar_drain, 0); ++spin) {}
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     const int slot = (warp - 2) / 4;                 // which tile of the pair
