@@ -13,6 +13,7 @@ step); the device time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -36,6 +37,34 @@ BF16_DATASHEET_TFLOPS = 2250.0
 FP8_OVER_BF16 = 2.0          # nominal dense FP8 / BF16 tensor throughput ratio
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNELS_PER_STEP = 6         # pool(Q), pool(K), pool(V), score, select, bsa
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one bsa_kernel launch, from
+# an ncu capture of that launch on the named workload (summaries under profiles/).  A figure
+# holds only for the kernel source it was taken on: KERNEL_SOURCES are hashed and compared.
+KERNEL_SOURCES = ("block_sparse_attention_oam_b200/csrc/stem_bsa.cu", "block_sparse_attention_oam_b200/csrc/stem_internal.cuh")
+MEASURED_TRAFFIC = {
+    # (workload, keep): (bytes per launch, sha256 of KERNEL_SOURCES, profile summary)
+    ("qwen3_8b_layer_s128k_fp8", 0.25): (2.24e9, "c2f06043d377e9038e3870812035576fc4f67e2767e0ba027dac6a711eff2a84",
+                                         "profiles/launches_s128k_fp8_keep25.md"),
+    ("qwen3_8b_layer_s64k_bf16", 0.25): (1.443e9, "c2f06043d377e9038e3870812035576fc4f67e2767e0ba027dac6a711eff2a84",
+                                         "profiles/bsa_kernel_bf16_s64k_keep25.md"),
+}
+
+
+def kernel_sha256() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(wl) -> float | None:
+    """Bytes per bsa_kernel launch measured on this workload with the current kernel source,
+    else None (another workload, or the kernel changed since the counters were taken)."""
+    rec = MEASURED_TRAFFIC.get((wl.name, wl.keep))
+    if rec is None or rec[1] != kernel_sha256():
+        return None
+    return rec[0]
 
 
 def measured_peaks():
@@ -375,7 +404,7 @@ def main():
         "effective_tflops": {"bsa": achieved, "prefill": flops_sel / (step_ms * 1e-3) / 1e12,
                              "bsa_frac_of_bf16_datasheet": achieved / BF16_DATASHEET_TFLOPS},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak, "traffic": measured_traffic(wl),
                      "peak_source": f"{peak_src} bf16_tflops_sustained" + (" x2 (fp8 nominal ratio)" if fp8 else ""),
                      "kernel": "bsa_kernel"},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
