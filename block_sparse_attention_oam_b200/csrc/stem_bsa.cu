@@ -341,11 +341,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
     if (lane == 0) {
       uint32_t itk[2] = {0, 0}, itv[2] = {0, 0}, gb[2] = {0, 0}, tq = 0;
       bool alive = true;
-      // S = Q K^T of the slot's next block into its S/P columns
-      auto issue_s = [&](int s, bool last) -> bool {
-        const uint32_t t = itk[s] % C::NST, ph = (itk[s] / C::NST) & 1;
-        if (!mbar_wait(k_full(s, t), ph, abort_flag, p.status)) return false;
-        tc_fence_after();
+      // S = Q K^T of a block (K in ring stage t) into the slot's S/P columns
+      auto issue_mmas_s = [&](int s, uint32_t t) {
         const uint32_t d_tmem = tmem + 256 * s;
 #pragma unroll
         for (int k = 0; k < C::S_KSTEPS; ++k) {
@@ -358,6 +355,13 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
           else
             mma_bf16(d_tmem, ad, bd, C::IDESC_S, k > 0);
         }
+      };
+      // the first S of a unit
+      auto issue_s = [&](int s, bool last) -> bool {
+        const uint32_t t = itk[s] % C::NST, ph = (itk[s] / C::NST) & 1;
+        if (!mbar_wait(k_full(s, t), ph, abort_flag, p.status)) return false;
+        tc_fence_after();
+        issue_mmas_s(s, t);
         mma_commit(s_full(s));
         mma_commit(k_empty(s, t));
         if (last) mma_commit(q_empty(s));  // every S of this unit issued: Q may be replaced
@@ -376,26 +380,56 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
         ++tq;
         for (int jj = 0; jj < n && alive; ++jj) {
           for (int s = 0; s < ns; ++s) {
+            // With two or more ring stages, V_j and K_{j+1} have landed long before P_j is
+            // ready: wait for them first, so that P V_j and S_{j+1} go out back to back as
+            // soon as P_j arrives.  With one stage K_{j+1} is only loaded once S_j is done,
+            // so P V_j goes first and the wait for K_{j+1} follows it.
+            constexpr bool kEarlyK = C::NST >= 2;
             const uint32_t t = itv[s] % C::NST, ph = (itv[s] / C::NST) & 1;
             if (!mbar_wait(v_full(s, t), ph, abort_flag, p.status)) { alive = false; break; }
+            const bool more = jj + 1 < n;
+            const uint32_t tk = itk[s] % C::NST, pk = (itk[s] / C::NST) & 1;
+            if (kEarlyK && more && !mbar_wait(k_full(s, tk), pk, abort_flag, p.status)) { alive = false; break; }
             if (!mbar_wait(p_full(s), gb[s] & 1, abort_flag, p.status)) { alive = false; break; }
             ++gb[s];
             tc_fence_after();
-            const uint32_t d_tmem = tmem + 256 * s + 128;
+            const uint32_t o_tmem = tmem + 256 * s + 128;
 #pragma unroll
             for (int k = 0; k < C::PV_KSTEPS; ++k) {
               const uint64_t bd =
                   smem_desc_sw128(sV + (s * C::NST + t) * C::KV_BYTES + k * C::PV_KROWS * 128, C::KV_CHUNK, 1024);
               const uint32_t acc = (jj > 0 || k > 0) ? 1u : 0u;
               if (FP8)
-                mma_fp8_ts(d_tmem, tmem + 256 * s + k * 8, bd, C::IDESC_PV, acc);
+                mma_fp8_ts(o_tmem, tmem + 256 * s + k * 8, bd, C::IDESC_PV, acc);
               else
-                mma_bf16_ts(d_tmem, tmem + 256 * s + k * 8, bd, C::IDESC_PV, acc);
+                mma_bf16_ts(o_tmem, tmem + 256 * s + k * 8, bd, C::IDESC_PV, acc);
             }
-            mma_commit(v_empty(s, t));
-            if (jj + 1 == n) mma_commit(o_done(s));
+            if (kEarlyK) {
+              // S_{j+1} straight behind P V_j; the commits follow
+              if (more) {
+                issue_mmas_s(s, tk);
+                mma_commit(s_full(s));
+              }
+              mma_commit(v_empty(s, t));
+              if (!more) mma_commit(o_done(s));
+            } else {
+              // one-stage ring: release V_j's stage as soon as P V_j completes, so that
+              // V_{j+1} loads while S_{j+1} runs
+              mma_commit(v_empty(s, t));
+              if (!more) mma_commit(o_done(s));
+              if (more) {
+                if (!mbar_wait(k_full(s, tk), pk, abort_flag, p.status)) { alive = false; break; }
+                tc_fence_after();
+                issue_mmas_s(s, tk);
+                mma_commit(s_full(s));
+              }
+            }
             ++itv[s];
-            if (jj + 1 < n && !issue_s(s, jj + 2 == n)) { alive = false; break; }
+            if (more) {
+              mma_commit(k_empty(s, tk));
+              if (jj + 2 == n) mma_commit(q_empty(s));  // the unit's last S: Q may be replaced
+              ++itk[s];
+            }
           }
         }
       }
