@@ -36,16 +36,16 @@ METRIC = "Stem prefill ms/layer at 128K, 25% budget; effective TFLOP/s vs B200 p
 BF16_DATASHEET_TFLOPS = 2250.0
 FP8_OVER_BF16 = 2.0          # nominal dense FP8 / BF16 tensor throughput ratio
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_STEP = 6         # pool(Q), pool(K), pool(V), score, select, bsa
+KERNELS_PER_STEP = 6         # pool(Q), pool(K), pool(V), score, select, bsa (+1 for FP8: its first-row bsa launch)
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one bsa_kernel launch, from
 # an ncu capture of that launch on the named workload (summaries under profiles/).  A figure
 # holds only for the kernel source it was taken on: KERNEL_SOURCES are hashed and compared.
 KERNEL_SOURCES = ("block_sparse_attention_oam_b200/csrc/stem_bsa.cu", "block_sparse_attention_oam_b200/csrc/stem_internal.cuh")
 MEASURED_TRAFFIC = {
-    # (workload, keep): (bytes per launch, sha256 of KERNEL_SOURCES, profile summary)
-    ("qwen3_8b_layer_s128k_fp8", 0.25): (2.24e9, "c2f06043d377e9038e3870812035576fc4f67e2767e0ba027dac6a711eff2a84",
+    # (workload, keep, mu, beta): (bytes per launch, sha256 of KERNEL_SOURCES, profile summary)
+    ("qwen3_8b_layer_s128k_fp8", 0.25, 0.7, 0.2): (2.24e9, "c2f06043d377e9038e3870812035576fc4f67e2767e0ba027dac6a711eff2a84",
                                          "profiles/launches_s128k_fp8_keep25.md"),
-    ("qwen3_8b_layer_s64k_bf16", 0.25): (1.443e9, "c2f06043d377e9038e3870812035576fc4f67e2767e0ba027dac6a711eff2a84",
+    ("qwen3_8b_layer_s64k_bf16", 0.25, 0.7, 0.2): (1.443e9, "c2f06043d377e9038e3870812035576fc4f67e2767e0ba027dac6a711eff2a84",
                                          "profiles/bsa_kernel_bf16_s64k_keep25.md"),
 }
 
@@ -61,7 +61,7 @@ def kernel_sha256() -> str:
 def measured_traffic(wl) -> float | None:
     """Bytes per bsa_kernel launch measured on this workload with the current kernel source,
     else None (another workload, or the kernel changed since the counters were taken)."""
-    rec = MEASURED_TRAFFIC.get((wl.name, wl.keep))
+    rec = MEASURED_TRAFFIC.get((wl.name, wl.keep, wl.mu, wl.beta))
     if rec is None or rec[1] != kernel_sha256():
         return None
     return rec[0]
@@ -286,16 +286,23 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default=W.LONG_128K_FP8.name, choices=sorted(W.ALL))
     ap.add_argument("--keep", type=float, default=None)
+    ap.add_argument("--mu", type=float, default=None, help="end-to-start budget ratio (1 = uniform budget)")
+    ap.add_argument("--beta", type=float, default=None, help="weight of the log-norm term (0 = routing score only)")
     ap.add_argument("--seqlen", type=int, default=None, help="replace the workload's sequences by one of this length")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
     ap.add_argument("--sweep", action="store_true", help="density sweep (keep 1.0 .. 0.1) against the dense kernel")
     args = ap.parse_args()
     wl = W.ALL[args.workload]
     if args.keep is not None:
         wl = wl.with_(keep=args.keep)
+    if args.mu is not None:
+        wl = wl.with_(mu=args.mu)
+    if args.beta is not None:
+        wl = wl.with_(beta=args.beta)
     if args.seqlen is not None:
         wl = wl.with_(seqlens=(args.seqlen,), name=f"{wl.name}@{args.seqlen}")
     if args.impl == "reference":
@@ -407,7 +414,7 @@ def main():
                      "frac": achieved / peak, "traffic": measured_traffic(wl),
                      "peak_source": f"{peak_src} bf16_tflops_sustained" + (" x2 (fp8 nominal ratio)" if fp8 else ""),
                      "kernel": "bsa_kernel"},
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": (KERNELS_PER_STEP + (1 if fp8 else 0)) * args.steps,
         "clocks": clk,
     }
 
@@ -424,6 +431,29 @@ def main():
         dense_ms = statistics.mean(dt)
         result["dense"] = {"bsa_dense_ms": dense_ms, "speedup_prefill_vs_dense": dense_ms / step_ms,
                            "dense_tflops": flops_dense / (dense_ms * 1e-3) / 1e12}
+        S.query_status(ws)
+
+    if not args.no_graph:
+        # the whole path (every kernel of stem_attention) replayed as one CUDA graph,
+        # inputs resident: what the per-call launch overhead costs
+        graph, _ = S.capture_attention(prob, q, k, v, paged, out=out, ws=ws)
+        for _ in range(2):
+            graph.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        g_ms = a.elapsed_time(b) / args.steps
+        if dist is not None:
+            t = torch.tensor([g_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            g_ms = float(t.item())
+        result["graph"] = {"ms_per_step": g_ms, "kernels_per_replay": KERNELS_PER_STEP + (1 if fp8 else 0),
+                           "note": "stem_attention captured in one CUDA graph, inputs resident"}
+        del graph
         S.query_status(ws)
 
     if not args.no_e2e:

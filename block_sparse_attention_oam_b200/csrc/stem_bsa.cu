@@ -107,22 +107,28 @@ struct Unit {
   bool two;          // the pair's second head exists
 };
 
+// Which units a launch covers.  kAllRows: every q-block row.  kRestRows: rows 1..N-1 of
+// every sequence; kFirstRow: row 0 only (FP8 runs the two, the first-row launch with the
+// two-term P; see the softmax).
+enum : int { kAllRows = 0, kRestRows = 1, kFirstRow = 2 };
+
 // Unit order: sequences by decreasing length; inside a sequence head pair by head pair,
 // rows from the last (longest list) to the first.  The CTAs running at one time then
 // share one pair's kv-head(s), whose K/V fit in L2.
+template <int PART>
 __device__ __forceinline__ Unit decode_unit(const BsaParams& p, int u) {
   Unit r{0, 0, 0, false};
   const int NP = (p.Hq + 1) / 2;
   int acc = 0;
   for (int q = 0; q < p.bt.num_seqs; ++q) {
     const int b = p.order[q];
-    const int nb = p.bt.seq[b].nblk;
+    const int nb = PART == kFirstRow ? 1 : (PART == kRestRows ? p.bt.seq[b].nblk - 1 : p.bt.seq[b].nblk);
     const int nu = nb * NP;
     if (u < acc + nu) {
       const int local = u - acc;
       const int pair = local / nb;
       r.b = b;
-      r.i = nb - 1 - (local - pair * nb);
+      r.i = PART == kFirstRow ? 0 : p.bt.seq[b].nblk - 1 - (local - pair * nb);
       r.h0 = 2 * pair;
       r.two = r.h0 + 1 < p.Hq;
       return r;
@@ -169,7 +175,7 @@ __device__ __forceinline__ const int32_t* head_list(const BsaParams& p, const Un
   return p.col_idx + static_cast<long long>(h) * p.bt.nnz_per_head + p.row_ptr[row];
 }
 
-template <int D, int BN, bool FP8, bool PAGED, bool DENSE>
+template <int D, int BN, bool FP8, bool PAGED, bool DENSE, int PART>
 __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant__ BsaParams p) {
   using C = Cfg<D, BN, FP8>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -235,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
     uint32_t itk[2] = {0, 0}, itv[2] = {0, 0}, tq = 0;
     bool alive = true;
     for (int u = blockIdx.x; u < p.total_units && alive; u += gridDim.x) {
-      const Unit un = decode_unit(p, u);
+      const Unit un = decode_unit<PART>(p, u);
       const int n = unit_len<DENSE>(p, un);
       if (n == 0) {
         if (lane == 0) atomicOr(p.status, kStatusBounds);
@@ -369,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
         return true;
       };
       for (int u = blockIdx.x; u < p.total_units && alive; u += gridDim.x) {
-        const Unit un = decode_unit(p, u);
+        const Unit un = decode_unit<PART>(p, u);
         const int n = unit_len<DENSE>(p, un);
         if (n == 0) continue;
         const int ns = un.two ? 2 : 1;
@@ -403,6 +409,15 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
                 mma_fp8_ts(o_tmem, tmem + 256 * s + k * 8, bd, C::IDESC_PV, acc);
               else
                 mma_bf16_ts(o_tmem, tmem + 256 * s + k * 8, bd, C::IDESC_PV, acc);
+            }
+            if constexpr (FP8 && PART == kFirstRow) {
+              // diagonal block: the residual term P_lo (columns P_COLS.. of the slot)
+#pragma unroll
+              for (int k = 0; k < C::PV_KSTEPS; ++k) {
+                const uint64_t bd =
+                    smem_desc_sw128(sV + (s * C::NST + t) * C::KV_BYTES + k * C::PV_KROWS * 128, C::KV_CHUNK, 1024);
+                mma_fp8_ts(o_tmem, tmem + 256 * s + C::P_COLS + k * 8, bd, C::IDESC_PV, 1u);
+              }
             }
             if (kEarlyK) {
               // S_{j+1} straight behind P V_j; the commits follow
@@ -450,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
     uint32_t gb = 0, ot = 0;                         // blocks and units processed by this slot
     bool alive = true;
     for (int u = blockIdx.x; u < p.total_units && alive; u += gridDim.x) {
-      const Unit un = decode_unit(p, u);
+      const Unit un = decode_unit<PART>(p, u);
       const int n = unit_len<DENSE>(p, un);
       if (n == 0 || (slot == 1 && !un.two)) continue;
       const int h = un.h0 + slot;
@@ -491,7 +506,11 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
           tq4[q] = make_float2(0.f, 0.f);
         }
         // P is packed in place over the first P_COLS registers of sr (each pair or quad of
-        // scores is read before its packed word is written)
+        // scores is read before its packed word is written).  FP8, diagonal block: P goes
+        // to the product as two e4m3 terms, P = P_hi + P_lo with P_lo the rounded residual
+        // of P_hi (stored after P_hi in TMEM and multiplied by V in a second product):
+        // the diagonal block holds the first rows of a sequence, whose few keys would
+        // otherwise carry e4m3's 2^-4 relative rounding straight into the output.
         auto exps = [&](auto want_lse) {
           if constexpr (!FP8) {
 #pragma unroll
@@ -519,6 +538,38 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
           exps(std::true_type{});
         else
           exps(std::false_type{});
+        if constexpr (FP8 && PART == kFirstRow) {
+          {
+            // residual pass (diagonal block only), before P_hi overwrites S in TMEM: S is
+            // read again 32 columns at a time into score registers the pass above freed
+            // (sr[64..95]); P_lo words go to sr[32..63] and then after P_hi in TMEM
+#pragma unroll
+            for (int c = 0; c < BN / 32; ++c) {
+              tmem_ld32(my_S + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+              tmem_wait_ld();
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                float x[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  x[e] = __uint_as_float(sr[64 + 4 * q + e]);
+                  if (c * 32 + 4 * q + e > r) x[e] = -INFINITY;
+                }
+                const float2 y0 = fma2(make_float2(x[0], x[1]), sc2, bias2);
+                const float2 y1 = fma2(make_float2(x[2], x[3]), sc2, bias2);
+                const uint32_t w = sr[8 * c + q];
+                const float2 h01 = e4m3x2_to_float2(static_cast<uint16_t>(w & 0xFFFFu));
+                const float2 h23 = e4m3x2_to_float2(static_cast<uint16_t>(w >> 16));
+                const float2 r0 = make_float2(ex2_approx(y0.x) - h01.x, ex2_approx(y0.y) - h01.y);
+                const float2 r1 = make_float2(ex2_approx(y1.x) - h23.x, ex2_approx(y1.y) - h23.y);
+                const uint32_t wl = __byte_perm(pack_e4m3x2(r0.x, r0.y), pack_e4m3x2(r1.x, r1.y), 0x5410);
+                sr[32 + 8 * c + q] = wl;
+                sq[q % 4] = add2(sq[q % 4], e4m3x4_pairsum(wl));
+              }
+            }
+            tmem_st32(my_S + C::P_COLS, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+          }
+        }
         const float2 sum2 = add2(add2(sq[0], sq[1]), add2(sq[2], sq[3]));
         const float2 sumt2 = add2(add2(tq4[0], tq4[1]), add2(tq4[2], tq4[3]));
         static_assert(C::P_COLS % 32 == 0, "P columns");
@@ -627,11 +678,11 @@ bool make_map(CUtensorMap* m, const void* ptr, bool fp8, int d, int H, long long
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int BN, bool FP8, bool PAGED, bool DENSE>
+template <int D, int BN, bool FP8, bool PAGED, bool DENSE, int PART>
 cudaError_t run(const BsaParams& prm, cudaStream_t st) {
   using C = Cfg<D, BN, FP8>;
-  auto kern = bsa_kernel<D, BN, FP8, PAGED, DENSE>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_LAUNCH);
+  auto kern = bsa_kernel<D, BN, FP8, PAGED, DENSE, PART>;
+  cudaError_t e = set_smem_once<bsa_kernel<D, BN, FP8, PAGED, DENSE, PART>>(C::SMEM_LAUNCH);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
@@ -642,10 +693,33 @@ cudaError_t run(const BsaParams& prm, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+template <int D, int BN, bool FP8, int PART>
+cudaError_t run_part(const BsaParams& prm, bool paged, bool dense, cudaStream_t st) {
+  if (paged)
+    return dense ? run<D, BN, FP8, true, true, PART>(prm, st) : run<D, BN, FP8, true, false, PART>(prm, st);
+  return dense ? run<D, BN, FP8, false, true, PART>(prm, st) : run<D, BN, FP8, false, false, PART>(prm, st);
+}
+
+// BF16: one launch over all rows.  FP8: rows 1.. in the main launch, then each sequence's
+// first q-block row (where rows have fewer keys than a block) in a small second launch.
 template <int D, int BN, bool FP8>
-cudaError_t run_mode(const BsaParams& prm, bool paged, bool dense, cudaStream_t st) {
-  if (paged) return dense ? run<D, BN, FP8, true, true>(prm, st) : run<D, BN, FP8, true, false>(prm, st);
-  return dense ? run<D, BN, FP8, false, true>(prm, st) : run<D, BN, FP8, false, false>(prm, st);
+cudaError_t run_mode(BsaParams prm, bool paged, bool dense, cudaStream_t st) {
+  const int NP = (prm.Hq + 1) / 2;
+  if constexpr (!FP8) {
+    long long units = 0;
+    for (int b = 0; b < prm.bt.num_seqs; ++b) units += static_cast<long long>(prm.bt.seq[b].nblk) * NP;
+    prm.total_units = static_cast<int>(units);
+    return run_part<D, BN, FP8, kAllRows>(prm, paged, dense, st);
+  } else {
+    long long rest = 0;
+    for (int b = 0; b < prm.bt.num_seqs; ++b) rest += static_cast<long long>(prm.bt.seq[b].nblk - 1) * NP;
+    prm.total_units = static_cast<int>(rest);
+    cudaError_t e = run_part<D, BN, FP8, kRestRows>(prm, paged, dense, st);
+    if (e != cudaSuccess) return e;
+    prm.total_units = prm.bt.num_seqs * NP;
+    prm.inject = 0;  // a test injection applies to the first launch only
+    return run_part<D, BN, FP8, kFirstRow>(prm, paged, dense, st);
+  }
 }
 
 }  // namespace
@@ -679,9 +753,6 @@ cudaError_t launch_bsa(const Batch& bt, const BsaArgs& a, bool fp8, bool paged, 
   prm.p_bias = fp8 ? 0.80735492205760410f : 0.0f;  // log2(1.75)
   // l is accumulated from the scaled, rounded P, so the V scale is all that remains
   prm.out_scale = fp8 ? a.v_scale : 1.0f;
-  long long units = 0;
-  for (int b = 0; b < bt.num_seqs; ++b) units += static_cast<long long>(bt.seq[b].nblk) * ((a.Hq + 1) / 2);
-  prm.total_units = static_cast<int>(units);
   // sequences by decreasing block count (longest rows first)
   int ord[STEM_MAX_SEQS];
   for (int b = 0; b < bt.num_seqs; ++b) ord[b] = b;

@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <atomic>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -48,6 +49,22 @@ struct WsLayout {
   size_t col_idx;      // int32 [Hq, nnz_per_head]
   size_t total;
 };
+
+// Raise a kernel's dynamic shared-memory limit once per device (the attribute outlives the
+// call; setting it once also keeps the launch path free of non-stream calls, so a whole
+// call can be captured into a CUDA graph).
+template <auto KERN>
+cudaError_t set_smem_once(int bytes) {
+  static std::atomic<uint64_t> done{0};  // one bit per device ordinal (mod 64)
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(KERN, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 // ------------------------------------------------------------ device helpers
 #if defined(__CUDACC__)

@@ -164,8 +164,7 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const Batch bt, const 
 cudaError_t launch_select(const Batch& bt, const float* scores, int Hq, int32_t* row_ptr, int32_t* col_idx,
                           uint32_t* status, cudaStream_t st) {
   const size_t smem = static_cast<size_t>(kWarps) * (256 + STEM_MAX_BLOCKS) * sizeof(uint32_t);
-  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = set_smem_once<select_kernel>(static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(bt.total_rows, (Hq + kWarps - 1) / kWarps);
   select_kernel<<<grid, kThreads, smem, st>>>(bt, scores, Hq, row_ptr, col_idx, status);

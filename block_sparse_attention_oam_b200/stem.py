@@ -255,6 +255,25 @@ def stem_attention(prob: Problem, q, k, v, paged: Optional[PagedKV] = None, out=
     return out
 
 
+def capture_attention(prob: Problem, q, k, v, paged: Optional[PagedKV] = None, out=None, lse=None, row_ptr=None,
+                      col_idx=None, ws=None):
+    """Capture one stem_attention call (pooling, scoring, selection, BSA: every kernel of
+    the path) into a CUDA graph on these buffers.  `graph.replay()` re-runs the whole path
+    on whatever the buffers hold at replay time, with one launch from the host.  The
+    problem (sequence lengths, heads, knobs) is fixed by the capture.  Returns (graph, out)."""
+    out = _out(prob, q, out)
+    ws = workspace(prob, q.device) if ws is None else ws
+    side = torch.cuda.Stream(device=q.device)
+    side.wait_stream(torch.cuda.current_stream(q.device))
+    with torch.cuda.stream(side):  # one eager call first: kernel attributes and the budget plan
+        stem_attention(prob, q, k, v, paged, out, lse, row_ptr, col_idx, ws)
+    torch.cuda.current_stream(q.device).wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        stem_attention(prob, q, k, v, paged, out, lse, row_ptr, col_idx, ws)
+    return graph, out
+
+
 def stem_attention_noalloc(prob: Problem, q, k, v, paged: Optional[PagedKV] = None, out=None, lse=None,
                            row_ptr=None, col_idx=None, status=None, stream=None):
     """stem_attention with the library's static scratch instead of a workspace
