@@ -205,6 +205,37 @@ def select_all(s: np.ndarray, k: np.ndarray) -> list:
     return [[select_row(s[h, i, : i + 1], i, int(k[i])) for i in range(N)] for h in range(H)]
 
 
+# ---------------------------------------------------------------------------
+# One selection per KV group — an extension of this library, not in the pages.
+# READING (own): the g q-heads that read one kv-head share one list per row.  The
+# group's score of block j in row i is the sum over its q-heads, in head order, of
+# their OAM scores, taken in float32 (the precision the device ranks in, so both
+# sides rank the same numbers; the positive factor 1/g of a mean would not change the
+# order).  Budget, forced blocks and tie rule are those of the per-head selection.
+# ---------------------------------------------------------------------------
+def group_scores(s: np.ndarray, g: int) -> np.ndarray:
+    """s [Hq,N,N] -> [Hq/g, N, N] float32: the g heads of each group summed left to right."""
+    Hq = s.shape[0]
+    s32 = np.asarray(s, dtype=np.float32)
+    out = np.empty((Hq // g,) + s.shape[1:], dtype=np.float32)
+    for kh in range(Hq // g):
+        acc = s32[kh * g].copy()
+        for t in range(1, g):
+            acc = np.add(acc, s32[kh * g + t], dtype=np.float32)
+        out[kh] = acc
+    return out
+
+
+def select_all_shared(s: np.ndarray, k: np.ndarray, g: int) -> list:
+    """s [Hq,N,N], k [N] -> lists[kh][i], one list per group of g q-heads."""
+    return select_all(group_scores(s, g).astype(np.float64), k)
+
+
+def expand_shared(lists_g: list, g: int) -> list:
+    """Per-group lists -> per-q-head lists (q-head h uses group h // g)."""
+    return [lists_g[h // g] for h in range(len(lists_g) * g)]
+
+
 def to_csr(lists_per_seq: list, Hq: int):
     """lists_per_seq[b][h][i] -> (row_ptr [R+1] int32, col_idx [Hq, nnz] int32).
     row_ptr is shared by all heads (the budget does not depend on the head)."""
@@ -250,13 +281,18 @@ def attend(q, k, v, lists, block: int, sigma: float, rows=None):
 
 
 def stem_sequence(q, k, v, block: int, keep: float, mu: float, beta: float, sigma: float,
-                  rows=None):
-    """The whole path for one sequence: pool -> score -> plan -> select -> attend."""
+                  rows=None, shared_lists: bool = False):
+    """The whole path for one sequence: pool -> score -> plan -> select -> attend.
+    shared_lists: one list per KV group (see select_all_shared)."""
     qbar, kbar, lbar = pool_mean(q, block), pool_mean(k, block), pool_log_norm(v, block)
     s = oam_scores(qbar, kbar, lbar, sigma, beta)
     N = qbar.shape[1]
     r, K, kk = tpd_plan(N, keep, mu)
-    lists = select_all(s, kk)
+    if shared_lists:
+        g = q.shape[1] // k.shape[1]
+        lists = expand_shared(select_all_shared(s, kk, g), g)
+    else:
+        lists = select_all(s, kk)
     out, lse = attend(q, k, v, lists, block, sigma, rows)
     return dict(qbar=qbar, kbar=kbar, lbar=lbar, scores=s, r_start=r, total=K, k=kk,
                 lists=lists, out=out, lse=lse)

@@ -268,3 +268,66 @@ def test_forced_only_row_by_hand():
     w = np.array([math.exp(float(q[t, 0] @ k[u, 0])) for u in keys])
     expect = sum(wi * v[u, 0] for wi, u in zip(w, keys)) / w.sum()
     assert np.allclose(out[t, 0], expect, atol=1e-13)
+
+
+# ------------------------------------------------------ one selection per KV group
+# (an extension of this library, not in the pages: group score = float32 sum of the
+# group's q-head scores, then the per-head selection rules)
+def test_shared_lists_group_of_one_is_the_per_head_selection():
+    rng = np.random.default_rng(21)
+    s = rng.standard_normal((3, 9, 9)).astype(np.float32).astype(np.float64)
+    k = O.tpd_plan(9, 0.4, 0.7)[2]
+    assert np.array_equal(O.group_scores(s, 1), s.astype(np.float32))
+    assert O.select_all_shared(s, k, 1) == O.select_all(s, k)
+
+
+def test_shared_lists_identical_heads_give_the_head_lists():
+    """Groups of identical heads (integer scores, so every float32 sum is exact): the group's
+    list is each member head's own list."""
+    rng = np.random.default_rng(22)
+    for g in (2, 3, 4):
+        base = rng.integers(-3, 4, size=(2, 10, 10)).astype(np.float64)
+        s = np.repeat(base, g, axis=0)
+        k = O.tpd_plan(10, 0.35, 0.7)[2]
+        shared = O.select_all_shared(s, k, g)
+        own = O.select_all(s, k)
+        for h in range(2 * g):
+            assert shared[h // g] == own[h]
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_shared_lists_brute_force_small(seed):
+    """Integer scores (exact sums in any order): every group list is the unique subset that
+    the (summed score descending, index ascending) order puts first."""
+    rng = np.random.default_rng(30 + seed)
+    g, N = 2, 8
+    s = rng.integers(-2, 3, size=(2 * g, N, N)).astype(np.float64)
+    k = O.tpd_plan(N, 0.45, 0.7)[2]
+    shared = O.select_all_shared(s, k, g)
+    for kh in range(2):
+        tot = sum(s[kh * g + t] for t in range(g))       # float64 sum of small integers: exact
+        for i in range(N):
+            got = shared[kh][i]
+            m = min(2, i + 1)
+            valid = [sorted({0, i} | set(c)) for c in itertools.combinations(range(1, i), int(k[i]) - m)]
+            winners = [c for c in valid if _dominance_ok(tot[i], i, c)]
+            assert len(winners) == 1 and got == winners[0]
+            assert got[0] == 0 and got[-1] == i and len(got) == k[i]
+
+
+def test_shared_lists_keep_one_is_dense_causal_attention():
+    rng = np.random.default_rng(23)
+    S, Hq, Hkv, d, B = 64, 4, 2, 8, 16
+    q, k, v = rng.standard_normal((S, Hq, d)), rng.standard_normal((S, Hkv, d)), rng.standard_normal((S, Hkv, d))
+    res = O.stem_sequence(q, k, v, B, 1.0, 0.7, 0.2, 0.3, shared_lists=True)
+    assert np.allclose(res["out"], _sdpa(q, k, v, 0.3, causal=True), atol=1e-12)
+
+
+def test_shared_lists_members_of_a_group_read_the_same_blocks():
+    rng = np.random.default_rng(24)
+    S, Hq, Hkv, d, B = 160, 8, 2, 8, 16                      # g = 4, 10 blocks
+    q, k, v = rng.standard_normal((S, Hq, d)), rng.standard_normal((S, Hkv, d)), rng.standard_normal((S, Hkv, d))
+    res = O.stem_sequence(q, k, v, B, 0.3, 0.7, 0.2, 0.3, shared_lists=True)
+    for h in range(Hq):
+        assert res["lists"][h] == res["lists"][(h // 4) * 4]
+        assert [len(r) for r in res["lists"][h]] == list(res["k"])
