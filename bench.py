@@ -61,7 +61,7 @@ def kernel_sha256() -> str:
 def measured_traffic(wl) -> float | None:
     """Bytes per bsa_kernel launch measured on this workload with the current kernel source,
     else None (another workload, or the kernel changed since the counters were taken)."""
-    rec = MEASURED_TRAFFIC.get((wl.name, wl.keep, wl.mu, wl.beta))
+    rec = None if wl.shared_lists else MEASURED_TRAFFIC.get((wl.name, wl.keep, wl.mu, wl.beta))
     if rec is None or rec[1] != kernel_sha256():
         return None
     return rec[0]
@@ -241,7 +241,7 @@ def run_sweep(args):
         ws = S.workspace(prob)
         scores = torch.empty((wl.num_q_heads, sz["scores_per_head"]), dtype=torch.float32, device="cuda")
         rp = torch.empty(sz["num_rows"] + 1, dtype=torch.int32, device="cuda")
-        ci = torch.empty((wl.num_q_heads, sz["nnz_per_head"]), dtype=torch.int32, device="cuda")
+        ci = torch.empty((sz["list_heads"], sz["nnz_per_head"]), dtype=torch.int32, device="cuda")
         out = torch.empty((sz["total_tokens"], wl.num_q_heads, wl.head_dim), dtype=torch.bfloat16, device="cuda")
         S.stem_score(prob, q, k, v, scores=scores, ws=ws)
         S.stem_select(prob, scores, rp, ci, ws=ws)
@@ -288,6 +288,8 @@ def main():
     ap.add_argument("--keep", type=float, default=None)
     ap.add_argument("--mu", type=float, default=None, help="end-to-start budget ratio (1 = uniform budget)")
     ap.add_argument("--beta", type=float, default=None, help="weight of the log-norm term (0 = routing score only)")
+    ap.add_argument("--shared-lists", action="store_true",
+                    help="one selection per KV group (an extension of this library, not in the pages)")
     ap.add_argument("--seqlen", type=int, default=None, help="replace the workload's sequences by one of this length")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -303,6 +305,8 @@ def main():
         wl = wl.with_(mu=args.mu)
     if args.beta is not None:
         wl = wl.with_(beta=args.beta)
+    if args.shared_lists:
+        wl = wl.with_(shared_lists=True)
     if args.seqlen is not None:
         wl = wl.with_(seqlens=(args.seqlen,), name=f"{wl.name}@{args.seqlen}")
     if args.impl == "reference":
@@ -339,7 +343,7 @@ def main():
     ws = S.workspace(prob)
     scores = torch.empty((wl.num_q_heads, sz["scores_per_head"]), dtype=torch.float32, device="cuda")
     rp = torch.empty(sz["num_rows"] + 1, dtype=torch.int32, device="cuda")
-    ci = torch.empty((wl.num_q_heads, sz["nnz_per_head"]), dtype=torch.int32, device="cuda")
+    ci = torch.empty((sz["list_heads"], sz["nnz_per_head"]), dtype=torch.int32, device="cuda")
     out = torch.empty((sz["total_tokens"], wl.num_q_heads, wl.head_dim), dtype=torch.bfloat16, device="cuda")
     stream = torch.cuda.current_stream()
 
@@ -402,7 +406,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "seq_len": list(wl.seqlens), "keep": wl.keep, "mu": wl.mu,
-                   "beta": wl.beta, "block": wl.block, "heads": [wl.num_q_heads, wl.num_kv_heads],
+                   "beta": wl.beta, "shared_lists": wl.shared_lists, "block": wl.block, "heads": [wl.num_q_heads, wl.num_kv_heads],
                    "head_dim": wl.head_dim, "paged": wl.paged, "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2 (no flush)"},
         "stages_ms": {"score": statistics.mean(st_score), "select": statistics.mean(st_select), "bsa": bsa_ms},

@@ -181,6 +181,8 @@ stem_status_t check_problem(const stem_problem_t* pr) {
   if (!(pr->mu > 0.0 && pr->mu <= 1.0)) return fail(STEM_ERR_INVALID, "mu %g outside (0, 1]", pr->mu);
   if (!std::isfinite(pr->beta)) return fail(STEM_ERR_INVALID, "beta is not finite");
   if (!std::isfinite(pr->softmax_scale)) return fail(STEM_ERR_INVALID, "softmax_scale is not finite");
+  if (pr->shared_lists != 0 && pr->shared_lists != 1)
+    return fail(STEM_ERR_INVALID, "shared_lists %d must be 0 or 1", pr->shared_lists);
   long long T = pr->cu_seqlens[pr->num_seqs];
   if (T > (1ll << 30)) return fail(STEM_ERR_UNSUPPORTED, "total tokens %lld too large", T);
   for (int b = 0; b < pr->num_seqs; ++b) {
@@ -240,6 +242,10 @@ void build_batch(const stem_problem_t* pr, Batch* bt) {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Lists of one selection: a list per q-head, or per KV group with shared lists.
+int list_heads(const stem_problem_t* pr) { return pr->shared_lists ? pr->num_kv_heads : pr->num_q_heads; }
+int list_group(const stem_problem_t* pr) { return pr->num_q_heads / list_heads(pr); }
+
 WsLayout layout(const stem_problem_t* pr, const Batch& bt) {
   WsLayout L;
   size_t o = 0;
@@ -257,7 +263,7 @@ WsLayout layout(const stem_problem_t* pr, const Batch& bt) {
   L.row_ptr = o;
   o = align256(o + (R + 1) * 4);
   L.col_idx = o;
-  o = align256(o + static_cast<size_t>(pr->num_q_heads) * static_cast<size_t>(bt.nnz_per_head) * 4);
+  o = align256(o + static_cast<size_t>(list_heads(pr)) * static_cast<size_t>(bt.nnz_per_head) * 4);
   L.total = o;
   return L;
 }
@@ -327,6 +333,7 @@ stem_status_t do_bsa(const stem_problem_t* pr, const Batch& bt, const WsLayout& 
   a.kv_rows = pg ? static_cast<long long>(pg->num_slots) * STEM_PAGE_SIZE : bt.total_tokens;
   a.row_ptr = row_ptr;
   a.col_idx = col_idx;
+  a.list_group = list_group(pr);
   a.out = out;
   a.lse = lse;
   a.Hq = pr->num_q_heads;
@@ -382,6 +389,7 @@ stem_status_t stem_query_sizes(const stem_problem_t* prob, stem_sizes_t* out) {
   out->nnz_per_head = bt.nnz_per_head;
   out->total_tokens = bt.total_tokens;
   out->workspace_bytes = L.total;
+  out->list_heads = list_heads(prob);
   return STEM_OK;
 }
 
@@ -423,8 +431,8 @@ stem_status_t stem_select(const stem_problem_t* prob, const float* scores, int32
   build_batch(prob, &bt);
   WsLayout L;
   if ((s = check_ws(prob, bt, ws, ws_bytes, &L)) != STEM_OK) return s;
-  cudaError_t e = launch_select(bt, scores, prob->num_q_heads, row_ptr, col_idx, at<uint32_t>(ws, L.status),
-                                static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_select(bt, scores, prob->num_q_heads, list_group(prob), row_ptr, col_idx,
+                                at<uint32_t>(ws, L.status), static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "select");
   return STEM_OK;
 }
@@ -477,7 +485,8 @@ stem_status_t stem_attention(const stem_problem_t* prob, const void* q, const vo
   int32_t* rp = at<int32_t>(ws, L.row_ptr);
   int32_t* ci = at<int32_t>(ws, L.col_idx);
   if ((s = do_score(prob, bt, L, q, k, v, paged, scores, ws, st)) != STEM_OK) return s;
-  cudaError_t e = launch_select(bt, scores, prob->num_q_heads, rp, ci, at<uint32_t>(ws, L.status), st);
+  cudaError_t e = launch_select(bt, scores, prob->num_q_heads, list_group(prob), rp, ci, at<uint32_t>(ws, L.status),
+                                st);
   if (e != cudaSuccess) return cuda_fail(e, "select");
   if ((s = do_bsa(prob, bt, L, q, k, v, paged, rp, ci, out, lse, ws, false, st)) != STEM_OK) return s;
   if (row_ptr_out != nullptr) {
@@ -485,7 +494,7 @@ stem_status_t stem_attention(const stem_problem_t* prob, const void* q, const vo
     if (e != cudaSuccess) return cuda_fail(e, "copy row_ptr");
   }
   if (col_idx_out != nullptr) {
-    e = cudaMemcpyAsync(col_idx_out, ci, static_cast<size_t>(prob->num_q_heads) * bt.nnz_per_head * 4,
+    e = cudaMemcpyAsync(col_idx_out, ci, static_cast<size_t>(list_heads(prob)) * bt.nnz_per_head * 4,
                         cudaMemcpyDeviceToDevice, st);
     if (e != cudaSuccess) return cuda_fail(e, "copy col_idx");
   }

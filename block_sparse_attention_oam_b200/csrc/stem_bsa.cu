@@ -86,6 +86,7 @@ struct BsaParams {
   Batch bt;
   const int32_t* row_ptr;
   const int32_t* col_idx;
+  int list_group;    // q-heads per list (1, or Hq/Hkv with shared lists)
   const int32_t* block_table;
   int max_pages;
   int num_slots;
@@ -172,7 +173,7 @@ __device__ __forceinline__ int unit_len(const BsaParams& p, const Unit& un) {
 }
 __device__ __forceinline__ const int32_t* head_list(const BsaParams& p, const Unit& un, int h) {
   const int row = p.bt.seq[un.b].row0 + un.i;
-  return p.col_idx + static_cast<long long>(h) * p.bt.nnz_per_head + p.row_ptr[row];
+  return p.col_idx + static_cast<long long>(h / p.list_group) * p.bt.nnz_per_head + p.row_ptr[row];
 }
 
 template <int D, int BN, bool FP8, bool PAGED, bool DENSE, int PART>
@@ -737,6 +738,7 @@ cudaError_t launch_bsa(const Batch& bt, const BsaArgs& a, bool fp8, bool paged, 
   prm.bt = bt;
   prm.row_ptr = a.row_ptr;
   prm.col_idx = a.col_idx;
+  prm.list_group = a.list_group > 0 ? a.list_group : 1;
   prm.block_table = a.block_table;
   prm.max_pages = a.max_pages;
   prm.num_slots = paged ? static_cast<int>(a.kv_rows / STEM_PAGE_SIZE) : 0;

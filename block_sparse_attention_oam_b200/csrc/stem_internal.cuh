@@ -405,8 +405,9 @@ cudaError_t launch_pool(const Batch& bt, const PoolArgs& a, int head_dim, bool f
                         cudaStream_t st);
 cudaError_t launch_score(const Batch& bt, const float* qbar, const float* kbar, const float* lbar, int Hq, int Hkv,
                          int head_dim, float sigma, float beta, float* scores, cudaStream_t st);
-cudaError_t launch_select(const Batch& bt, const float* scores, int Hq, int32_t* row_ptr, int32_t* col_idx,
-                          uint32_t* status, cudaStream_t st);
+// group = q-heads per list (1: a list per q-head; Hq/Hkv: a list per KV group)
+cudaError_t launch_select(const Batch& bt, const float* scores, int Hq, int group, int32_t* row_ptr,
+                          int32_t* col_idx, uint32_t* status, cudaStream_t st);
 
 struct BsaArgs {
   const void* q;
@@ -417,6 +418,7 @@ struct BsaArgs {
   long long kv_rows;        // rows of the K/V tensor maps (T, or num_slots * page)
   const int32_t* row_ptr;   // nullptr in dense mode
   const int32_t* col_idx;
+  int list_group;           // q-heads per list: 1, or Hq/Hkv with shared lists
   void* out;
   float* lse;
   int Hq, Hkv, head_dim;

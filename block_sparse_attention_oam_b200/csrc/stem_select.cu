@@ -9,9 +9,11 @@
 //  * section "用架构师的眼睛看稀疏注意力": the initial tokens are the trunk every
 //    output depends on, so block 0 is always kept (and so is the diagonal block).
 //
-// One CTA per (global block row, group of 8 q-heads).  The CTA recomputes the
-// row's budget k_i and its CSR offset sum_{i'<i} k_i' from r_start (fp64, the same
-// operation order as the host planner), then each warp selects one head's row:
+// One CTA per (global block row, group of 8 lists).  The CTA recomputes the row's
+// budget k_i and its CSR offset sum_{i'<i} k_i' from r_start (fp64, the same
+// operation order as the host planner), then each warp selects one list's row (a
+// list per q-head, or — shared lists, an extension of this library — a list per KV
+// group ranked by the float32 sum, in head order, of its q-heads' scores):
 // a most-significant-digit-first radix select (4 passes of 8 bits, histogram in
 // shared memory) finds the k-th largest order-preserving score key, and a
 // ballot-based compaction walks the candidates in ascending block order, taking
@@ -34,7 +36,7 @@ __device__ __forceinline__ uint32_t score_key(float f) {
 }
 
 __global__ void __launch_bounds__(kThreads) select_kernel(const Batch bt, const float* __restrict__ scores,
-                                                          int Hq, int32_t* __restrict__ row_ptr,
+                                                          int Hq, int group, int32_t* __restrict__ row_ptr,
                                                           int32_t* __restrict__ col_idx, uint32_t* status) {
   extern __shared__ uint32_t sm[];
   uint32_t* hist_all = sm;                              // [kWarps][256]
@@ -68,8 +70,8 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const Batch bt, const 
     if (b == bt.num_seqs - 1 && i == N - 1) row_ptr[row + 1] = static_cast<int32_t>(s.nnz0 + off + k_i);
   }
 
-  const int h = blockIdx.y * kWarps + warp;
-  if (h >= Hq) return;
+  const int h = blockIdx.y * kWarps + warp;  // list index
+  if (h >= Hq / group) return;
   int32_t* out = col_idx + static_cast<long long>(h) * bt.nnz_per_head + s.nnz0 + off;
   const unsigned full = 0xffffffffu;
   if (i == 0) {
@@ -90,11 +92,15 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const Batch bt, const 
     return;
   }
 
-  const float* srow = scores + static_cast<long long>(h) * bt.scores_per_head + s.score0 +
+  const float* srow = scores + static_cast<long long>(h) * group * bt.scores_per_head + s.score0 +
                       static_cast<long long>(i) * (i + 1) / 2;
   uint32_t* keys = keys_all + warp * STEM_MAX_BLOCKS;
   uint32_t* hist = hist_all + warp * 256;
-  for (int j = 1 + lane; j < i; j += 32) keys[j] = score_key(srow[j]);
+  for (int j = 1 + lane; j < i; j += 32) {
+    float v = srow[j];
+    for (int t = 1; t < group; ++t) v = __fadd_rn(v, srow[static_cast<long long>(t) * bt.scores_per_head + j]);
+    keys[j] = score_key(v);
+  }
   __syncwarp();
 
   uint32_t prefix = 0, pmask = 0;
@@ -161,13 +167,13 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const Batch bt, const 
 
 }  // namespace
 
-cudaError_t launch_select(const Batch& bt, const float* scores, int Hq, int32_t* row_ptr, int32_t* col_idx,
-                          uint32_t* status, cudaStream_t st) {
+cudaError_t launch_select(const Batch& bt, const float* scores, int Hq, int group, int32_t* row_ptr,
+                          int32_t* col_idx, uint32_t* status, cudaStream_t st) {
   const size_t smem = static_cast<size_t>(kWarps) * (256 + STEM_MAX_BLOCKS) * sizeof(uint32_t);
   cudaError_t e = set_smem_once<select_kernel>(static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  dim3 grid(bt.total_rows, (Hq + kWarps - 1) / kWarps);
-  select_kernel<<<grid, kThreads, smem, st>>>(bt, scores, Hq, row_ptr, col_idx, status);
+  dim3 grid(bt.total_rows, (Hq / group + kWarps - 1) / kWarps);
+  select_kernel<<<grid, kThreads, smem, st>>>(bt, scores, Hq, group, row_ptr, col_idx, status);
   return cudaGetLastError();
 }
 

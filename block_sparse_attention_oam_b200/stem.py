@@ -46,6 +46,7 @@ class _Problem(ctypes.Structure):
         ("beta", ctypes.c_float),
         ("keep", ctypes.c_double),
         ("mu", ctypes.c_double),
+        ("shared_lists", ctypes.c_int),
     ]
 
 
@@ -67,6 +68,7 @@ class _Sizes(ctypes.Structure):
         ("nnz_per_head", ctypes.c_int64),
         ("total_tokens", ctypes.c_int64),
         ("workspace_bytes", ctypes.c_size_t),
+        ("list_heads", ctypes.c_int64),
     ]
 
 
@@ -138,6 +140,7 @@ class Problem:
     beta: float = 0.2
     keep: float = 0.25
     mu: float = 0.7
+    shared_lists: bool = False   # one selection per KV group (an extension, not in the pages)
 
     def __post_init__(self):
         self._cu = np.ascontiguousarray(np.asarray(self.cu_seqlens, dtype=np.int32))
@@ -145,7 +148,7 @@ class Problem:
                            self.num_q_heads, self.num_kv_heads, self.head_dim, self.block_size,
                            DT_FP8 if self.dtype == "fp8_e4m3" else DT_BF16,
                            self.q_scale, self.k_scale, self.v_scale, self.softmax_scale, self.beta,
-                           self.keep, self.mu)
+                           self.keep, self.mu, 1 if self.shared_lists else 0)
 
     @property
     def c(self):
@@ -155,7 +158,7 @@ class Problem:
         s = _Sizes()
         _check(lib().stem_query_sizes(self.c, ctypes.byref(s)))
         return dict(num_rows=s.num_rows, scores_per_head=s.scores_per_head, nnz_per_head=s.nnz_per_head,
-                    total_tokens=s.total_tokens, workspace_bytes=s.workspace_bytes)
+                    total_tokens=s.total_tokens, workspace_bytes=s.workspace_bytes, list_heads=s.list_heads)
 
 
 @dataclasses.dataclass
@@ -215,7 +218,7 @@ def stem_select(prob: Problem, scores, row_ptr=None, col_idx=None, ws=None, stre
     if row_ptr is None:
         row_ptr = torch.empty(sz["num_rows"] + 1, dtype=torch.int32, device=dev)
     if col_idx is None:
-        col_idx = torch.empty((prob.num_q_heads, sz["nnz_per_head"]), dtype=torch.int32, device=dev)
+        col_idx = torch.empty((sz["list_heads"], sz["nnz_per_head"]), dtype=torch.int32, device=dev)
     ws = workspace(prob, dev) if ws is None else ws
     _check(lib().stem_select(prob.c, _ptr(scores), _ptr(row_ptr), _ptr(col_idx), _ptr(ws), ws.numel(),
                              _stream(stream)))
@@ -306,4 +309,4 @@ def problem_for(wl, inputs=None, keep=None) -> Problem:
     if inputs is not None and wl.dtype == "fp8_e4m3":
         kw = dict(q_scale=inputs.q_scale, k_scale=inputs.k_scale, v_scale=inputs.v_scale)
     return Problem(cu, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.block, wl.dtype, beta=wl.beta,
-                   keep=wl.keep if keep is None else keep, mu=wl.mu, **kw)
+                   keep=wl.keep if keep is None else keep, mu=wl.mu, shared_lists=wl.shared_lists, **kw)

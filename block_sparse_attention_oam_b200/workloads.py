@@ -40,6 +40,7 @@ class Workload:
     page_size: int = 64
     style: str = "qwen"          # "tiny" or "qwen": value distribution recipe
     seed: int = 0
+    shared_lists: bool = False   # one selection per KV group (an extension, not in the pages)
 
     @property
     def total_tokens(self) -> int:

@@ -74,6 +74,11 @@ typedef struct {
   float beta;                  /* OAM weight of the log||V|| term (0.2 in the article) */
   double keep;                 /* fraction of causal block pairs kept, in (0, 1] */
   double mu;                   /* TPD end-to-start keep ratio (0.7 in the article), in (0, 1] */
+  int shared_lists;            /* 0: one selection per q-head (the article's method).
+                                  1: one selection per KV group — an extension of this library,
+                                  not in the pages: the group's score of a block is the float32
+                                  sum, in head order, of its q-heads' OAM scores; every q-head of
+                                  the group uses the group's list (col_idx then has Hkv rows). */
 } stem_problem_t;
 
 /* Optional paged KV cache (vLLM style).  Pass NULL for contiguous K/V. */
@@ -93,6 +98,7 @@ typedef struct {
   int64_t nnz_per_head;        /* sum_b K_b: selected (q-block, kv-block) pairs per q-head */
   int64_t total_tokens;        /* T */
   size_t workspace_bytes;      /* device workspace for any entry point of this problem */
+  int64_t list_heads;          /* rows of col_idx: Hq, or Hkv with shared_lists */
 } stem_sizes_t;
 
 /* Sizes of every buffer of the problem.  Host only.  Returns STEM_ERR_* on a bad problem. */
@@ -138,8 +144,10 @@ STEM_API stem_status_t stem_score(const stem_problem_t* prob, const void* q, con
  * scores: DEVICE float [Hq, scores_per_head] (layout of stem_score).
  * row_ptr: DEVICE int32 [num_rows + 1], shared by all heads (the budget does not
  *   depend on the head); row (b, i) is global row sum_{b'<b} N_b' + i.
- * col_idx: DEVICE int32 [Hq, nnz_per_head]: ascending block indices local to
- *   the sequence, diagonal last; head h's row r is col_idx[h*nnz + row_ptr[r] ...].
+ * col_idx: DEVICE int32 [list_heads, nnz_per_head]: ascending block indices
+ *   local to the sequence, diagonal last; list l's row r is
+ *   col_idx[l*nnz + row_ptr[r] ...].  list_heads = Hq (list l = q-head l) or, with
+ *   shared_lists, Hkv (list l = KV group l, ranked by the group's summed scores).
  */
 STEM_API stem_status_t stem_select(const stem_problem_t* prob, const float* scores, int32_t* row_ptr,
                           int32_t* col_idx, void* ws, size_t ws_bytes, void* stream);
@@ -149,6 +157,8 @@ STEM_API stem_status_t stem_select(const stem_problem_t* prob, const float* scor
  * (q-head, q-block) the kernel walks only the listed KV blocks with an online
  * softmax and no per-block branch; skipped blocks behave exactly as if all their
  * scores were -inf; only the diagonal block is token-masked.
+ * col_idx: [list_heads, nnz_per_head] as stem_select writes it; q-head h walks list
+ *   h / (Hq / list_heads).
  * out: DEVICE bf16 [T, Hq, d].  lse: DEVICE float [Hq, T] natural-log
  * log-sum-exp of sigma*q.k over the visited keys, or NULL.
  * FP8: Q/K/V are e4m3 codes with per-tensor scales; P is rounded to e4m3 for

@@ -99,3 +99,17 @@ def test_entry_points_reject_before_launch(L):
     assert st == S.STEM_ERR_INVALID
     assert b"NULL" in L.stem_last_error()
     assert L.stem_status_string(S.STEM_ERR_TIMEOUT) == b"device pipeline wait timed out"
+
+
+def test_shared_lists_sizes_and_validation(L):
+    """One selection per KV group: col_idx has Hkv rows; any other flag value is refused."""
+    cu = np.array([0, 1024, 3000])
+    per_head = S.Problem(cu, 8, 2, 128, 128).sizes()
+    shared = S.Problem(cu, 8, 2, 128, 128, shared_lists=True).sizes()
+    assert per_head["list_heads"] == 8 and shared["list_heads"] == 2
+    assert shared["nnz_per_head"] == per_head["nnz_per_head"]
+    assert shared["workspace_bytes"] < per_head["workspace_bytes"]
+    p = S.Problem(cu, 8, 2, 128, 128)
+    p._c.shared_lists = 2
+    st = L.stem_query_sizes(p.c, ctypes.byref(S._Sizes()))
+    assert st == S.STEM_ERR_INVALID
