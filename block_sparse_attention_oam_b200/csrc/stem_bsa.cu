@@ -176,7 +176,7 @@ __device__ __forceinline__ const int32_t* head_list(const BsaParams& p, const Un
   return p.col_idx + static_cast<long long>(h / p.list_group) * p.bt.nnz_per_head + p.row_ptr[row];
 }
 
-template <int D, int BN, bool FP8, bool PAGED, bool DENSE, int PART>
+template <int D, int BN, bool FP8, bool PAGED, bool DENSE, int PART, bool SHKV>
 __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant__ BsaParams p) {
   using C = Cfg<D, BN, FP8>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -199,6 +199,15 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
   auto p_full = [&](int s) { return b0 + 192 * s + 152; };
   auto o_done = [&](int s) { return b0 + 192 * s + 160; };
   const uint32_t bar_drain = b0 + 384;
+  // K/V rings.  Per slot: NST stages each.  SHKV (both tiles of a pair walk one list of one
+  // kv-head): one ring of 2*NST stages over both slots' memory, each tile loaded once and
+  // released after both slots' products (empty barriers expect two arrivals).
+  constexpr int RING = SHKV ? 2 * C::NST : C::NST;
+  auto kv_off = [&](int s, uint32_t t) { return (SHKV ? t : s * C::NST + t) * C::KV_BYTES; };
+  auto kf = [&](int s, uint32_t t) { return SHKV ? k_full(t / C::NST, t % C::NST) : k_full(s, t); };
+  auto ke = [&](int s, uint32_t t) { return SHKV ? k_empty(t / C::NST, t % C::NST) : k_empty(s, t); };
+  auto vf = [&](int s, uint32_t t) { return SHKV ? v_full(t / C::NST, t % C::NST) : v_full(s, t); };
+  auto ve = [&](int s, uint32_t t) { return SHKV ? v_empty(t / C::NST, t % C::NST) : v_empty(s, t); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_area + 448);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_area + 456);
 
@@ -209,9 +218,9 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
       mbar_init(q_empty(s), 1);
       for (int t = 0; t < C::NST; ++t) {
         mbar_init(k_full(s, t), 1);
-        mbar_init(k_empty(s, t), 1);
+        mbar_init(k_empty(s, t), SHKV ? 2 : 1);
         mbar_init(v_full(s, t), 1);
-        mbar_init(v_empty(s, t), 1);
+        mbar_init(v_empty(s, t), SHKV ? 2 : 1);
       }
       mbar_init(s_full(s), 1);
       mbar_init(p_full(s), 4);
@@ -302,28 +311,30 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
             for (int hh = 0; hh < C::HALVES; ++hh) rows[s][hh] = __shfl_sync(full, rowh[s][hh], q);
           for (int s = 0; s < ns; ++s) {
             const int kvh = (un.h0 + s) / G;
-            const uint32_t t = itk[s] % C::NST, ph = (itk[s] / C::NST) & 1;
-            if (!warp_wait(k_empty(s, t), ph ^ 1, abort_flag, p.status)) { alive = false; break; }
+            if (SHKV && s > 0) break;  // one copy of the shared tile
+            const uint32_t t = itk[s] % RING, ph = (itk[s] / RING) & 1;
+            if (!warp_wait(ke(s, t), ph ^ 1, abort_flag, p.status)) { alive = false; break; }
             const bool withhold = p.inject == 1 && blockIdx.x == 0 && s == 0 && itk[0] == 0;
             if (lane == 0 && !withhold) {
-              mbar_arrive_expect_tx(k_full(s, t), C::KV_BYTES);
+              mbar_arrive_expect_tx(kf(s, t), C::KV_BYTES);
               for (int c = 0; c < C::DCH; ++c)
                 for (int hh = 0; hh < C::HALVES; ++hh)
-                  tma_load_3d(sK + (s * C::NST + t) * C::KV_BYTES + c * C::KV_CHUNK + hh * 64 * 128, &p.tk,
-                              k_full(s, t), c * C::CH, kvh, rows[s][hh]);
+                  tma_load_3d(sK + kv_off(s, t) + c * C::KV_CHUNK + hh * 64 * 128, &p.tk, kf(s, t), c * C::CH,
+                              kvh, rows[s][hh]);
             }
             ++itk[s];
           }
           for (int s = 0; s < ns && alive; ++s) {
             const int kvh = (un.h0 + s) / G;
-            const uint32_t t = itv[s] % C::NST, ph = (itv[s] / C::NST) & 1;
-            if (!warp_wait(v_empty(s, t), ph ^ 1, abort_flag, p.status)) { alive = false; break; }
+            if (SHKV && s > 0) break;
+            const uint32_t t = itv[s] % RING, ph = (itv[s] / RING) & 1;
+            if (!warp_wait(ve(s, t), ph ^ 1, abort_flag, p.status)) { alive = false; break; }
             if (lane == 0) {
-              mbar_arrive_expect_tx(v_full(s, t), C::KV_BYTES);
+              mbar_arrive_expect_tx(vf(s, t), C::KV_BYTES);
               for (int c = 0; c < C::DCH; ++c)
                 for (int hh = 0; hh < C::HALVES; ++hh)
-                  tma_load_3d(sV + (s * C::NST + t) * C::KV_BYTES + c * C::KV_CHUNK + hh * 64 * 128, &p.tv,
-                              v_full(s, t), c * C::CH, kvh, rows[s][hh]);
+                  tma_load_3d(sV + kv_off(s, t) + c * C::KV_CHUNK + hh * 64 * 128, &p.tv, vf(s, t), c * C::CH,
+                              kvh, rows[s][hh]);
             }
             ++itv[s];
           }
@@ -333,10 +344,10 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
     if (!alive) {
       // let the copies already issued land before the CTA can exit
       for (int s = 0; s < 2; ++s) {
-        for (uint32_t q = (itk[s] > C::NST ? itk[s] - C::NST : 0); q < itk[s]; ++q)
-          for (int spin = 0; spin < 1000000 && !mbar_try_wait(k_full(s, q % C::NST), (q / C::NST) & 1); ++spin) {}
-        for (uint32_t q = (itv[s] > C::NST ? itv[s] - C::NST : 0); q < itv[s]; ++q)
-          for (int spin = 0; spin < 1000000 && !mbar_try_wait(v_full(s, q % C::NST), (q / C::NST) & 1); ++spin) {}
+        for (uint32_t q = (itk[s] > RING ? itk[s] - RING : 0); q < itk[s]; ++q)
+          for (int spin = 0; spin < 1000000 && !mbar_try_wait(kf(s, q % RING), (q / RING) & 1); ++spin) {}
+        for (uint32_t q = (itv[s] > RING ? itv[s] - RING : 0); q < itv[s]; ++q)
+          for (int spin = 0; spin < 1000000 && !mbar_try_wait(vf(s, q % RING), (q / RING) & 1); ++spin) {}
       }
       if (tq > 0)
         for (int s = 0; s < 2; ++s)
@@ -356,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
           const int c = k / 4, w = k % 4;
           const uint64_t ad = smem_desc_sw128(sQ + s * C::Q_BYTES + c * C::Q_CHUNK + w * 32, 16, 1024);
           const uint64_t bd =
-              smem_desc_sw128(sK + (s * C::NST + t) * C::KV_BYTES + c * C::KV_CHUNK + w * 32, 16, 1024);
+              smem_desc_sw128(sK + kv_off(s, t) + c * C::KV_CHUNK + w * 32, 16, 1024);
           if (FP8)
             mma_fp8(d_tmem, ad, bd, C::IDESC_S, k > 0);
           else
@@ -365,12 +376,12 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
       };
       // the first S of a unit
       auto issue_s = [&](int s, bool last) -> bool {
-        const uint32_t t = itk[s] % C::NST, ph = (itk[s] / C::NST) & 1;
-        if (!mbar_wait(k_full(s, t), ph, abort_flag, p.status)) return false;
+        const uint32_t t = itk[s] % RING, ph = (itk[s] / RING) & 1;
+        if (!mbar_wait(kf(s, t), ph, abort_flag, p.status)) return false;
         tc_fence_after();
         issue_mmas_s(s, t);
         mma_commit(s_full(s));
-        mma_commit(k_empty(s, t));
+        mma_commit(ke(s, t));
         if (last) mma_commit(q_empty(s));  // every S of this unit issued: Q may be replaced
         ++itk[s];
         return true;
@@ -391,12 +402,12 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
             // ready: wait for them first, so that P V_j and S_{j+1} go out back to back as
             // soon as P_j arrives.  With one stage K_{j+1} is only loaded once S_j is done,
             // so P V_j goes first and the wait for K_{j+1} follows it.
-            constexpr bool kEarlyK = C::NST >= 2;
-            const uint32_t t = itv[s] % C::NST, ph = (itv[s] / C::NST) & 1;
-            if (!mbar_wait(v_full(s, t), ph, abort_flag, p.status)) { alive = false; break; }
+            constexpr bool kEarlyK = RING >= 2;
+            const uint32_t t = itv[s] % RING, ph = (itv[s] / RING) & 1;
+            if (!mbar_wait(vf(s, t), ph, abort_flag, p.status)) { alive = false; break; }
             const bool more = jj + 1 < n;
-            const uint32_t tk = itk[s] % C::NST, pk = (itk[s] / C::NST) & 1;
-            if (kEarlyK && more && !mbar_wait(k_full(s, tk), pk, abort_flag, p.status)) { alive = false; break; }
+            const uint32_t tk = itk[s] % RING, pk = (itk[s] / RING) & 1;
+            if (kEarlyK && more && !mbar_wait(kf(s, tk), pk, abort_flag, p.status)) { alive = false; break; }
             if (!mbar_wait(p_full(s), gb[s] & 1, abort_flag, p.status)) { alive = false; break; }
             ++gb[s];
             tc_fence_after();
@@ -404,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
 #pragma unroll
             for (int k = 0; k < C::PV_KSTEPS; ++k) {
               const uint64_t bd =
-                  smem_desc_sw128(sV + (s * C::NST + t) * C::KV_BYTES + k * C::PV_KROWS * 128, C::KV_CHUNK, 1024);
+                  smem_desc_sw128(sV + kv_off(s, t) + k * C::PV_KROWS * 128, C::KV_CHUNK, 1024);
               const uint32_t acc = (jj > 0 || k > 0) ? 1u : 0u;
               if (FP8)
                 mma_fp8_ts(o_tmem, tmem + 256 * s + k * 8, bd, C::IDESC_PV, acc);
@@ -416,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
 #pragma unroll
               for (int k = 0; k < C::PV_KSTEPS; ++k) {
                 const uint64_t bd =
-                    smem_desc_sw128(sV + (s * C::NST + t) * C::KV_BYTES + k * C::PV_KROWS * 128, C::KV_CHUNK, 1024);
+                    smem_desc_sw128(sV + kv_off(s, t) + k * C::PV_KROWS * 128, C::KV_CHUNK, 1024);
                 mma_fp8_ts(o_tmem, tmem + 256 * s + C::P_COLS + k * 8, bd, C::IDESC_PV, 1u);
               }
             }
@@ -426,15 +437,15 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
                 issue_mmas_s(s, tk);
                 mma_commit(s_full(s));
               }
-              mma_commit(v_empty(s, t));
+              mma_commit(ve(s, t));
               if (!more) mma_commit(o_done(s));
             } else {
               // one-stage ring: release V_j's stage as soon as P V_j completes, so that
               // V_{j+1} loads while S_{j+1} runs
-              mma_commit(v_empty(s, t));
+              mma_commit(ve(s, t));
               if (!more) mma_commit(o_done(s));
               if (more) {
-                if (!mbar_wait(k_full(s, tk), pk, abort_flag, p.status)) { alive = false; break; }
+                if (!mbar_wait(kf(s, tk), pk, abort_flag, p.status)) { alive = false; break; }
                 tc_fence_after();
                 issue_mmas_s(s, tk);
                 mma_commit(s_full(s));
@@ -442,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
             }
             ++itv[s];
             if (more) {
-              mma_commit(k_empty(s, tk));
+              mma_commit(ke(s, tk));
               if (jj + 2 == n) mma_commit(q_empty(s));  // the unit's last S: Q may be replaced
               ++itk[s];
             }
@@ -679,11 +690,11 @@ bool make_map(CUtensorMap* m, const void* ptr, bool fp8, int d, int H, long long
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int BN, bool FP8, bool PAGED, bool DENSE, int PART>
+template <int D, int BN, bool FP8, bool PAGED, bool DENSE, int PART, bool SHKV = false>
 cudaError_t run(const BsaParams& prm, cudaStream_t st) {
   using C = Cfg<D, BN, FP8>;
-  auto kern = bsa_kernel<D, BN, FP8, PAGED, DENSE, PART>;
-  cudaError_t e = set_smem_once<bsa_kernel<D, BN, FP8, PAGED, DENSE, PART>>(C::SMEM_LAUNCH);
+  auto kern = bsa_kernel<D, BN, FP8, PAGED, DENSE, PART, SHKV>;
+  cudaError_t e = set_smem_once<bsa_kernel<D, BN, FP8, PAGED, DENSE, PART, SHKV>>(C::SMEM_LAUNCH);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
@@ -696,6 +707,12 @@ cudaError_t run(const BsaParams& prm, cudaStream_t st) {
 
 template <int D, int BN, bool FP8, int PART>
 cudaError_t run_part(const BsaParams& prm, bool paged, bool dense, cudaStream_t st) {
+  // shared lists with an even group size: both heads of every pair walk one list of one
+  // kv-head, so their K/V tiles are loaded once (instantiated for d = 128, block 128)
+  if constexpr (D == 128 && BN == 128) {
+    if (!dense && prm.list_group % 2 == 0)
+      return paged ? run<D, BN, FP8, true, false, PART, true>(prm, st) : run<D, BN, FP8, false, false, PART, true>(prm, st);
+  }
   if (paged)
     return dense ? run<D, BN, FP8, true, true, PART>(prm, st) : run<D, BN, FP8, true, false, PART>(prm, st);
   return dense ? run<D, BN, FP8, false, true, PART>(prm, st) : run<D, BN, FP8, false, false, PART>(prm, st);
