@@ -17,7 +17,8 @@
 namespace stem {
 namespace {
 
-constexpr int kPoolThreads = 128;
+constexpr int kPoolThreads = 128;   // threads across the token row (16 bytes each)
+constexpr int kPoolGroups = 4;      // token groups per block (more bytes in flight per CTA)
 
 __device__ __forceinline__ void decode16(const uint4& u, float* f, bool fp8, float scale) {
   if (!fp8) {
@@ -46,10 +47,12 @@ __device__ __forceinline__ void decode16(const uint4& u, float* f, bool fp8, flo
 }
 
 // One CTA per (global block row, group of 128 x VEC elements of the [H*d] token row).
-// Each thread owns VEC consecutive elements (16 bytes) of one head and walks the
-// block's tokens, so every warp reads 512 contiguous bytes per token.
+// Each thread owns VEC consecutive elements (16 bytes) of one head; the block's tokens
+// are split among kPoolGroups groups of 128 threads (contiguous quarters), so every warp
+// reads 512 contiguous bytes per token and a CTA keeps four token streams in flight.
+// The groups' partial sums are added in group order (deterministic).
 template <int D, bool FP8, bool PAGED>
-__global__ void __launch_bounds__(kPoolThreads) pool_kernel(const Batch bt, PoolArgs a) {
+__global__ void __launch_bounds__(kPoolThreads * kPoolGroups) pool_kernel(const Batch bt, PoolArgs a) {
   constexpr int VEC = FP8 ? 16 : 8;
   constexpr int LPH = D / VEC;  // lanes per head
   const int row = blockIdx.x;
@@ -61,7 +64,8 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const Batch bt, Pool
   const int t_end = min(s.len, t_beg + B);
   const int n = t_end - t_beg;
   const int HD = a.H * D;
-  const int e0 = (blockIdx.y * kPoolThreads + threadIdx.x) * VEC;
+  const int tx = threadIdx.x % kPoolThreads, grp = threadIdx.x / kPoolThreads;
+  const int e0 = (blockIdx.y * kPoolThreads + tx) * VEC;
   const bool valid = e0 < HD;
   const int h = valid ? e0 / D : 0;
   const int d0 = e0 % D;
@@ -85,12 +89,15 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const Batch bt, Pool
   };
 
   constexpr int U = 4;
-  for (int t = t_beg; t < t_end; t += U) {
+  const int chunk = (B + kPoolGroups - 1) / kPoolGroups;
+  const int g_beg = t_beg + grp * chunk;
+  const int g_end = min(t_end, g_beg + chunk);
+  for (int t = g_beg; t < g_end; t += U) {
     uint4 buf[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       buf[u] = make_uint4(0, 0, 0, 0);
-      if (valid && t + u < t_end) buf[u] = __ldg(tok_ptr(t + u));
+      if (valid && t + u < g_end) buf[u] = __ldg(tok_ptr(t + u));
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -105,11 +112,24 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const Batch bt, Pool
       if (a.lognorm_out != nullptr) {
 #pragma unroll
         for (int o = LPH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o, LPH);
-        if (t + u < t_end) lacc += logf(fmaxf(sqrtf(ss), FLT_MIN));
+        if (t + u < g_end) lacc += logf(fmaxf(sqrtf(ss), FLT_MIN));
       }
     }
   }
-  if (!valid) return;
+  // partial sums of groups 1.. to group 0, added in group order
+  __shared__ float part[kPoolGroups - 1][VEC + 1][kPoolThreads];
+  if (grp > 0) {
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) part[grp - 1][e][tx] = acc[e];
+    part[grp - 1][VEC][tx] = lacc;
+  }
+  __syncthreads();
+  if (grp > 0 || !valid) return;
+  for (int g = 0; g < kPoolGroups - 1; ++g) {
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) acc[e] += part[g][e][tx];
+    lacc += part[g][VEC][tx];
+  }
   const float inv = 1.0f / static_cast<float>(n);
   if (a.mean_out != nullptr) {
     float* dst = a.mean_out + (static_cast<long long>(h) * bt.total_rows + row) * D + d0;
@@ -126,9 +146,9 @@ cudaError_t pool_dispatch_paged(const Batch& bt, const PoolArgs& a, bool paged, 
   constexpr int VEC = FP8 ? 16 : 8;
   dim3 grid(bt.total_rows, (a.H * D + kPoolThreads * VEC - 1) / (kPoolThreads * VEC));
   if (paged)
-    pool_kernel<D, FP8, true><<<grid, kPoolThreads, 0, st>>>(bt, a);
+    pool_kernel<D, FP8, true><<<grid, kPoolThreads * kPoolGroups, 0, st>>>(bt, a);
   else
-    pool_kernel<D, FP8, false><<<grid, kPoolThreads, 0, st>>>(bt, a);
+    pool_kernel<D, FP8, false><<<grid, kPoolThreads * kPoolGroups, 0, st>>>(bt, a);
   return cudaGetLastError();
 }
 
