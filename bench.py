@@ -43,9 +43,9 @@ KERNELS_PER_STEP = 6         # pool(Q), pool(K), pool(V), score, select, bsa (+1
 KERNEL_SOURCES = ("block_sparse_attention_oam_b200/csrc/stem_bsa.cu", "block_sparse_attention_oam_b200/csrc/stem_internal.cuh")
 MEASURED_TRAFFIC = {
     # (workload, keep, mu, beta): (bytes per launch, sha256 of KERNEL_SOURCES, profile summary)
-    ("qwen3_8b_layer_s128k_fp8", 0.25, 0.7, 0.2): (2.24e9, "e4a8afb08c8965f148dbf2b40474cee7dad5cd8f8408c39c3dd93a3d20f091de",
+    ("qwen3_8b_layer_s128k_fp8", 0.25, 0.7, 0.2): (2.26e9, "55b04ddd543081fdcae47af260d3958606e9ff10ae5c171a8cbe480772e7ac4f",
                                          "profiles/launches_s128k_fp8_keep25.md"),
-    ("qwen3_8b_layer_s64k_bf16", 0.25, 0.7, 0.2): (1.444e9, "e4a8afb08c8965f148dbf2b40474cee7dad5cd8f8408c39c3dd93a3d20f091de",
+    ("qwen3_8b_layer_s64k_bf16", 0.25, 0.7, 0.2): (1.445e9, "55b04ddd543081fdcae47af260d3958606e9ff10ae5c171a8cbe480772e7ac4f",
                                          "profiles/bsa_kernel_bf16_s64k_keep25.md"),
 }
 
