@@ -176,7 +176,7 @@ __device__ __forceinline__ const int32_t* head_list(const BsaParams& p, const Un
   return p.col_idx + static_cast<long long>(h / p.list_group) * p.bt.nnz_per_head + p.row_ptr[row];
 }
 
-template <int D, int BN, bool FP8, bool PAGED, bool DENSE, int PART, bool SHKV>
+template <int D, int BN, bool FP8, bool PAGED, bool DENSE, int PART, bool SHKV, bool LSEX>
 __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant__ BsaParams p) {
   using C = Cfg<D, BN, FP8>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -546,10 +546,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
             }
           }
         };
-        if (FP8 && p.lse != nullptr)
-          exps(std::true_type{});
-        else
-          exps(std::false_type{});
+        // LSEX (FP8 with a log-sum-exp requested): also the sums of the unrounded P
+        exps(std::bool_constant<LSEX>{});
         if constexpr (FP8 && PART == kFirstRow) {
           {
             // residual pass (diagonal block only), before P_hi overwrites S in TMEM: S is
@@ -589,7 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
         for (int c = 0; c < C::P_COLS / 32; ++c) tmem_st32(my_S + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
         const float2 a2 = make_float2(alpha, alpha);
         l2 = fma2(l2, a2, sum2);
-        if (FP8) lt2 = fma2(lt2, a2, sumt2);
+        if constexpr (LSEX) lt2 = fma2(lt2, a2, sumt2);
         if (jj > 0 && __any_sync(full, resc)) {
           // O holds the sum up to the previous block: S_j was issued after P V_{j-1},
           // the tensor core runs in order, and S_j is complete
@@ -644,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
         }
       }
       if (p.lse != nullptr && r < rows_valid) {
-        const float lt = FP8 ? (lt2.x + lt2.y) / p.p_scale : l;
+        const float lt = LSEX ? (lt2.x + lt2.y) / p.p_scale : l;
         p.lse[static_cast<long long>(h) * p.bt.total_tokens + tok] = (m_run + __log2f(lt)) * 0.69314718055994531f;
       }
       tc_fence_before();
@@ -690,11 +688,11 @@ bool make_map(CUtensorMap* m, const void* ptr, bool fp8, int d, int H, long long
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int BN, bool FP8, bool PAGED, bool DENSE, int PART, bool SHKV = false>
-cudaError_t run(const BsaParams& prm, cudaStream_t st) {
+template <int D, int BN, bool FP8, bool PAGED, bool DENSE, int PART, bool SHKV, bool LSEX>
+cudaError_t run_k(const BsaParams& prm, cudaStream_t st) {
   using C = Cfg<D, BN, FP8>;
-  auto kern = bsa_kernel<D, BN, FP8, PAGED, DENSE, PART, SHKV>;
-  cudaError_t e = set_smem_once<bsa_kernel<D, BN, FP8, PAGED, DENSE, PART, SHKV>>(C::SMEM_LAUNCH);
+  auto kern = bsa_kernel<D, BN, FP8, PAGED, DENSE, PART, SHKV, LSEX>;
+  cudaError_t e = set_smem_once<bsa_kernel<D, BN, FP8, PAGED, DENSE, PART, SHKV, LSEX>>(C::SMEM_LAUNCH);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
@@ -703,6 +701,16 @@ cudaError_t run(const BsaParams& prm, cudaStream_t st) {
   if (grid <= 0) return cudaSuccess;
   kern<<<grid, kThreads, C::SMEM_LAUNCH, st>>>(prm);
   return cudaGetLastError();
+}
+
+// FP8 with a log-sum-exp requested keeps the unrounded P sums as well (its own kernel, so
+// the default one carries none of that work)
+template <int D, int BN, bool FP8, bool PAGED, bool DENSE, int PART, bool SHKV = false>
+cudaError_t run(const BsaParams& prm, cudaStream_t st) {
+  if constexpr (FP8) {
+    if (prm.lse != nullptr) return run_k<D, BN, FP8, PAGED, DENSE, PART, SHKV, true>(prm, st);
+  }
+  return run_k<D, BN, FP8, PAGED, DENSE, PART, SHKV, false>(prm, st);
 }
 
 template <int D, int BN, bool FP8, int PART>
