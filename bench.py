@@ -43,9 +43,9 @@ KERNELS_PER_STEP = 6         # pool(Q), pool(K), pool(V), score, select, bsa (+1
 KERNEL_SOURCES = ("block_sparse_attention_oam_b200/csrc/stem_bsa.cu", "block_sparse_attention_oam_b200/csrc/stem_internal.cuh")
 MEASURED_TRAFFIC = {
     # (workload, keep, mu, beta): (bytes per launch, sha256 of KERNEL_SOURCES, profile summary)
-    ("qwen3_8b_layer_s128k_fp8", 0.25, 0.7, 0.2): (2.26e9, "55b04ddd543081fdcae47af260d3958606e9ff10ae5c171a8cbe480772e7ac4f",
+    ("qwen3_8b_layer_s128k_fp8", 0.25, 0.7, 0.2): (2.25e9, "5cfb0402a236d8dcc3452ef1fc42d89c5d4eac767a53809bdf94a691741bee80",
                                          "profiles/launches_s128k_fp8_keep25.md"),
-    ("qwen3_8b_layer_s64k_bf16", 0.25, 0.7, 0.2): (1.445e9, "55b04ddd543081fdcae47af260d3958606e9ff10ae5c171a8cbe480772e7ac4f",
+    ("qwen3_8b_layer_s64k_bf16", 0.25, 0.7, 0.2): (1.442e9, "5cfb0402a236d8dcc3452ef1fc42d89c5d4eac767a53809bdf94a691741bee80",
                                          "profiles/bsa_kernel_bf16_s64k_keep25.md"),
 }
 
