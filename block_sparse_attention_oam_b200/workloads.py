@@ -94,44 +94,71 @@ def _rng(seed: int, stream: int) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, stream])))
 
 
+def _trng(seed: int, stream: int) -> torch.Generator:
+    """Seeded torch CPU generator for (workload seed, stream)."""
+    return torch.Generator().manual_seed((int(seed) * 1_000_003 + int(stream)) & 0x7FFFFFFFFFFFFFFF)
+
+
 def _unit_rows(rng, n, d):
     u = rng.standard_normal((n, d))
     return u / np.linalg.norm(u, axis=-1, keepdims=True)
 
 
-def _gen_sequence(wl: Workload, seq_index: int, S: int):
-    """Return float32 arrays q [S,Hq,d], k [S,Hkv,d], v [S,Hkv,d] for one sequence."""
+_CHUNK = 4096   # tokens generated per step (small float32 buffers, reused)
+
+
+def _gen_sequence_into(wl: Workload, seq_index: int, S: int, q_out, k_out, v_out) -> None:
+    """Fill bf16 tensors q_out [S,Hq,d], k_out [S,Hkv,d], v_out [S,Hkv,d] for one sequence,
+    _CHUNK tokens at a time (only the bf16 results are ever held at full size).
+    Q, K ~ N(0,1)/sqrt(d) with a sink bias on the first 128 keys; V rows of norm
+    sqrt(d) * exp(N(0, 0.5)) ("tiny": unit Q/K, a x4 sink direction on the first 64 keys,
+    V rows scaled by exp(N(0, 0.5)))."""
     d, Hq, Hkv = wl.head_dim, wl.num_q_heads, wl.num_kv_heads
     base = 16 * seq_index
-    rq, rk, rv, rn, ru = (_rng(wl.seed, base + i) for i in range(5))
-    q = rq.standard_normal((S, Hq, d), dtype=np.float32)
-    k = rk.standard_normal((S, Hkv, d), dtype=np.float32)
-    v = rv.standard_normal((S, Hkv, d), dtype=np.float32)
-    log_norm = rn.normal(0.0, 0.5, size=(S, Hkv)).astype(np.float32)
-    u = _unit_rows(ru, Hkv, d).astype(np.float32)            # sink direction per KV head
-    if wl.style == "tiny":
-        # keys of the first block share one direction (x4); V rows scaled by exp(N(0, 0.5))
-        nsink = min(64, S)
-        k[:nsink] += 4.0 * u[None, :, :]
-        v *= np.exp(log_norm)[:, :, None]
-    else:
-        # Q, K ~ N(0,1)/sqrt(d); sink bias on the first 128 keys; V rows of norm
-        # sqrt(d) * exp(N(0, 0.5)).
-        inv = np.float32(1.0 / math.sqrt(d))
-        q *= inv
-        k *= inv
-        nsink = min(128, S)
-        k[:nsink] += (4.0 * inv) * u[None, :, :]
-        v /= np.linalg.norm(v, axis=-1, keepdims=True)
-        v *= (math.sqrt(d) * np.exp(log_norm))[:, :, None]
-    return q, k, v
+    rn, ru = (_rng(wl.seed, base + i) for i in (3, 4))
+    gq, gk, gv = (_trng(wl.seed, base + i) for i in (0, 1, 2))
+    log_norm = torch.from_numpy(rn.normal(0.0, 0.5, size=(S, Hkv)).astype(np.float32))
+    u = torch.from_numpy(_unit_rows(ru, Hkv, d).astype(np.float32))   # sink direction per KV head
+    tiny = wl.style == "tiny"
+    inv = 1.0 if tiny else 1.0 / math.sqrt(d)
+    nsink = min(64 if tiny else 128, S)
+    sink = (4.0 if tiny else 4.0 * inv) * u
+    n0 = min(_CHUNK, S)
+    bq = torch.empty((n0, Hq, d), dtype=torch.float32)
+    bk = torch.empty((n0, Hkv, d), dtype=torch.float32)
+    bv = torch.empty((n0, Hkv, d), dtype=torch.float32)
+    for t0 in range(0, S, _CHUNK):
+        n = min(_CHUNK, S - t0)
+        q, k, v = bq[:n], bk[:n], bv[:n]
+        torch.randn((n, Hq, d), generator=gq, out=q)
+        torch.randn((n, Hkv, d), generator=gk, out=k)
+        torch.randn((n, Hkv, d), generator=gv, out=v)
+        if not tiny:
+            q.mul_(inv)
+            k.mul_(inv)
+        if t0 < nsink:
+            k[: nsink - t0] += sink[None, :, :]
+        ln = log_norm[t0: t0 + n]
+        if tiny:
+            v.mul_(torch.exp(ln)[:, :, None])
+        else:
+            v.div_(torch.linalg.vector_norm(v, dim=-1, keepdim=True))
+            v.mul_((math.sqrt(d) * torch.exp(ln))[:, :, None])
+        q_out[t0: t0 + n].copy_(q)
+        k_out[t0: t0 + n].copy_(k)
+        v_out[t0: t0 + n].copy_(v)
 
 
 def _quant_fp8(x_bf16: torch.Tensor):
-    amax = float(x_bf16.float().abs().max())
-    # a float32-representable scale, so host (float64) and device (float32) agree exactly
+    """Per-tensor e4m3 codes and scale (amax / 448, a float32-representable value, so host
+    float64 and device float32 agree exactly), a chunk of rows at a time."""
+    amax = 0.0
+    for t0 in range(0, x_bf16.shape[0], _CHUNK):
+        amax = max(amax, float(x_bf16[t0: t0 + _CHUNK].abs().max()))
     scale = float(np.float32(amax / FP8_E4M3_MAX)) if amax > 0 else 1.0
-    codes = (x_bf16.float() / scale).to(torch.float8_e4m3fn)
+    codes = torch.empty(x_bf16.shape, dtype=torch.float8_e4m3fn)
+    for t0 in range(0, x_bf16.shape[0], _CHUNK):
+        codes[t0: t0 + _CHUNK] = (x_bf16[t0: t0 + _CHUNK].float() / scale).to(torch.float8_e4m3fn)
     return codes, scale
 
 
@@ -139,16 +166,13 @@ def make_inputs(wl: Workload) -> Inputs:
     seqlens = [int(s) for s in wl.seqlens]
     cu = np.zeros(len(seqlens) + 1, dtype=np.int32)
     cu[1:] = np.cumsum(seqlens)
-    qs, ks, vs = [], [], []
+    T = int(cu[-1])
+    q = torch.empty((T, wl.num_q_heads, wl.head_dim), dtype=torch.bfloat16)
+    k = torch.empty((T, wl.num_kv_heads, wl.head_dim), dtype=torch.bfloat16)
+    v = torch.empty((T, wl.num_kv_heads, wl.head_dim), dtype=torch.bfloat16)
     for b, S in enumerate(seqlens):
-        q, k, v = _gen_sequence(wl, b, S)
-        qs.append(torch.from_numpy(q).to(torch.bfloat16))
-        ks.append(torch.from_numpy(k).to(torch.bfloat16))
-        vs.append(torch.from_numpy(v).to(torch.bfloat16))
-        del q, k, v
-    q = torch.cat(qs) if len(qs) > 1 else qs[0]
-    k = torch.cat(ks) if len(ks) > 1 else ks[0]
-    v = torch.cat(vs) if len(vs) > 1 else vs[0]
+        t0, t1 = int(cu[b]), int(cu[b + 1])
+        _gen_sequence_into(wl, b, S, q[t0:t1], k[t0:t1], v[t0:t1])
     inp = Inputs(wl, cu, q, k, v)
     if wl.dtype == "fp8_e4m3":
         inp.q, inp.q_scale = _quant_fp8(q)
