@@ -39,13 +39,15 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 KERNELS_PER_STEP = 6         # pool(Q), pool(K), pool(V), score, select, bsa (+1 for FP8: its first-row bsa launch)
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one bsa_kernel launch, from
 # an ncu capture of that launch on the named workload (summaries under profiles/).  A figure
-# holds only for the kernel source it was taken on: KERNEL_SOURCES are hashed and compared.
-KERNEL_SOURCES = ("block_sparse_attention_oam_b200/csrc/stem_bsa.cu", "block_sparse_attention_oam_b200/csrc/stem_internal.cuh")
+# holds only for the kernel source and the input generator it was taken on: KERNEL_SOURCES
+# are hashed and compared.
+KERNEL_SOURCES = ("block_sparse_attention_oam_b200/csrc/stem_bsa.cu", "block_sparse_attention_oam_b200/csrc/stem_internal.cuh",
+                  "block_sparse_attention_oam_b200/workloads.py")
 MEASURED_TRAFFIC = {
     # (workload, keep, mu, beta): (bytes per launch, sha256 of KERNEL_SOURCES, profile summary)
-    ("qwen3_8b_layer_s128k_fp8", 0.25, 0.7, 0.2): (2.25e9, "5cfb0402a236d8dcc3452ef1fc42d89c5d4eac767a53809bdf94a691741bee80",
+    ("qwen3_8b_layer_s128k_fp8", 0.25, 0.7, 0.2): (2.25e9, "c160b0e6d223bf018583022003436225313b22abc7dde071b2ce047e46e1fa9a",
                                          "profiles/launches_s128k_fp8_keep25.md"),
-    ("qwen3_8b_layer_s64k_bf16", 0.25, 0.7, 0.2): (1.442e9, "5cfb0402a236d8dcc3452ef1fc42d89c5d4eac767a53809bdf94a691741bee80",
+    ("qwen3_8b_layer_s64k_bf16", 0.25, 0.7, 0.2): (1.441e9, "c160b0e6d223bf018583022003436225313b22abc7dde071b2ce047e46e1fa9a",
                                          "profiles/bsa_kernel_bf16_s64k_keep25.md"),
 }
 
