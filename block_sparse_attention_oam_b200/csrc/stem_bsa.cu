@@ -94,6 +94,7 @@ struct BsaParams {
   float* lse;
   int Hq, Hkv;
   int total_units;   // sum over sequences of N_b * ceil(Hq / 2)
+  int groups;        // (sequence, head pair) groups with at least one unit in this launch
   float scale_log2;  // sigma * q_scale * k_scale * log2(e)
   float p_bias;      // log2 of the factor P is scaled by before rounding (FP8: log2 1.75)
   float out_scale;   // FP8: v_scale (l carries the P factor); BF16: 1
@@ -114,8 +115,12 @@ struct Unit {
 enum : int { kAllRows = 0, kRestRows = 1, kFirstRow = 2 };
 
 // Unit order: sequences by decreasing length; inside a sequence head pair by head pair,
-// rows from the last (longest list) to the first.  The CTAs running at one time then
-// share one pair's kv-head(s), whose K/V fit in L2.
+// so that the CTAs running at one time share one pair's kv-head(s), whose K/V fit in L2.
+// The rows of a group run alternately from the last (longest list) to the first and back,
+// the final group longest first: list lengths then change smoothly from unit to unit, and
+// the round-robin split over the CTAs gives each nearly the same number of blocks (a row
+// order that restarts at the longest row in every group leaves the first CTAs with the
+// longest row of every round).
 template <int PART>
 __device__ __forceinline__ Unit decode_unit(const BsaParams& p, int u) {
   Unit r{0, 0, 0, false};
@@ -128,8 +133,10 @@ __device__ __forceinline__ Unit decode_unit(const BsaParams& p, int u) {
     if (u < acc + nu) {
       const int local = u - acc;
       const int pair = local / nb;
+      const int pos = local - pair * nb;
+      const bool longest_first = ((p.groups - 1 - (q * NP + pair)) & 1) == 0;
       r.b = b;
-      r.i = PART == kFirstRow ? 0 : p.bt.seq[b].nblk - 1 - (local - pair * nb);
+      r.i = PART == kFirstRow ? 0 : (longest_first ? p.bt.seq[b].nblk - 1 - pos : p.bt.seq[b].nblk - nb + pos);
       r.h0 = 2 * pair;
       r.two = r.h0 + 1 < p.Hq;
       return r;
@@ -735,14 +742,19 @@ cudaError_t run_mode(BsaParams prm, bool paged, bool dense, cudaStream_t st) {
     long long units = 0;
     for (int b = 0; b < prm.bt.num_seqs; ++b) units += static_cast<long long>(prm.bt.seq[b].nblk) * NP;
     prm.total_units = static_cast<int>(units);
+    prm.groups = prm.bt.num_seqs * NP;
     return run_part<D, BN, FP8, kAllRows>(prm, paged, dense, st);
   } else {
     long long rest = 0;
     for (int b = 0; b < prm.bt.num_seqs; ++b) rest += static_cast<long long>(prm.bt.seq[b].nblk - 1) * NP;
     prm.total_units = static_cast<int>(rest);
+    int busy = 0;  // sequences with rows after the first (ordered first)
+    for (int b = 0; b < prm.bt.num_seqs; ++b) busy += prm.bt.seq[b].nblk > 1 ? 1 : 0;
+    prm.groups = busy * NP;
     cudaError_t e = run_part<D, BN, FP8, kRestRows>(prm, paged, dense, st);
     if (e != cudaSuccess) return e;
     prm.total_units = prm.bt.num_seqs * NP;
+    prm.groups = prm.bt.num_seqs * NP;
     prm.inject = 0;  // a test injection applies to the first launch only
     return run_part<D, BN, FP8, kFirstRow>(prm, paged, dense, st);
   }
