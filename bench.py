@@ -45,9 +45,9 @@ KERNEL_SOURCES = ("block_sparse_attention_oam_b200/csrc/stem_bsa.cu", "block_spa
                   "block_sparse_attention_oam_b200/workloads.py")
 MEASURED_TRAFFIC = {
     # (workload, keep, mu, beta): (bytes per launch, sha256 of KERNEL_SOURCES, profile summary)
-    ("qwen3_8b_layer_s128k_fp8", 0.25, 0.7, 0.2): (2.14e9, "be7ca89682d80e1f72efc3787e832cabbe722bfab6f5c507c93586a1cb9df067",
+    ("qwen3_8b_layer_s128k_fp8", 0.25, 0.7, 0.2): (2.14e9, "0faad37df4b9e65bfff87e4099340736e40601ecb236c8f7db3406492db9a144",
                                          "profiles/launches_s128k_fp8_keep25.md"),
-    ("qwen3_8b_layer_s64k_bf16", 0.25, 0.7, 0.2): (1.410e9, "be7ca89682d80e1f72efc3787e832cabbe722bfab6f5c507c93586a1cb9df067",
+    ("qwen3_8b_layer_s64k_bf16", 0.25, 0.7, 0.2): (1.409e9, "0faad37df4b9e65bfff87e4099340736e40601ecb236c8f7db3406492db9a144",
                                          "profiles/bsa_kernel_bf16_s64k_keep25.md"),
 }
 

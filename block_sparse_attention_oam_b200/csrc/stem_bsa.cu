@@ -540,6 +540,11 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
               sq[u2 % 4] = add2(sq[u2 % 4], make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
             }
           } else {
+            // sums of the rounded P: the e4m3 weights (exact in f16) go into two f16x2
+            // accumulators, one weight per lane and quad (relative rounding 2^-11 per
+            // addition), which are added in f32 every 16 quads — fewer conversions and
+            // shorter dependency chains on the exponential phase than a per-quad f32 sum
+            uint32_t hs[2] = {0u, 0u};
 #pragma unroll
             for (int u4 = 0; u4 < BN / 4; ++u4) {
               const float2 y0 = fma2(make_float2(__uint_as_float(sr[4 * u4]), __uint_as_float(sr[4 * u4 + 1])), sc2, bias2);
@@ -548,7 +553,18 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
               const float2 e1 = make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
               const uint32_t w = __byte_perm(pack_e4m3x2(e0.x, e0.y), pack_e4m3x2(e1.x, e1.y), 0x5410);
               sr[u4] = w;
-              sq[u4 % 4] = add2(sq[u4 % 4], e4m3x4_pairsum(w));
+              {
+                uint32_t a, b;
+                asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(a) : "h"(static_cast<uint16_t>(w & 0xFFFFu)));
+                asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(b) : "h"(static_cast<uint16_t>(w >> 16)));
+                hs[0] = hadd2_u32(hs[0], a);
+                hs[1] = hadd2_u32(hs[1], b);
+              }
+              if (u4 % 16 == 15) {
+                sq[(u4 / 16) % 4] = add2(sq[(u4 / 16) % 4], add2(h2_to_float2(hs[0]), h2_to_float2(hs[1])));
+                hs[0] = 0u;
+                hs[1] = 0u;
+              }
               if constexpr (decltype(want_lse)::value) tq4[u4 % 4] = add2(tq4[u4 % 4], add2(e0, e1));
             }
           }

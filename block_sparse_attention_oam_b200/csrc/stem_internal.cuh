@@ -321,18 +321,33 @@ __device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t v) {
   return make_float2(lo, hi);
 }
 
-// Four e4m3 codes (bytes 0..3) -> (b0 + b2, b1 + b3) as floats, the pair sums taken in f16.
-__device__ __forceinline__ float2 e4m3x4_pairsum(uint32_t v) {
-  uint32_t a, b, c;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(a) : "h"(static_cast<uint16_t>(v & 0xFFFFu)));
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(b) : "h"(static_cast<uint16_t>(v >> 16)));
+// Packed f16 pair addition.
+__device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b) {
+  uint32_t c;
   asm("add.rn.f16x2 %0, %1, %2;" : "=r"(c) : "r"(a), "r"(b));
+  return c;
+}
+
+// An f16x2 word -> two floats (low half first).
+__device__ __forceinline__ float2 h2_to_float2(uint32_t c) {
   float lo, hi;
   asm("{\n\t.reg .f16 x, y;\n\tmov.b32 {x, y}, %2;\n\tcvt.f32.f16 %0, x;\n\tcvt.f32.f16 %1, y;\n\t}\n"
       : "=f"(lo), "=f"(hi)
       : "r"(c));
   return make_float2(lo, hi);
 }
+
+// Four e4m3 codes (bytes 0..3) -> (b0 + b2, b1 + b3) as an f16x2 word: every e4m3 value is
+// exact in f16, the pair sums are rounded to f16.
+__device__ __forceinline__ uint32_t e4m3x4_pairsum_h(uint32_t v) {
+  uint32_t a, b;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(a) : "h"(static_cast<uint16_t>(v & 0xFFFFu)));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(b) : "h"(static_cast<uint16_t>(v >> 16)));
+  return hadd2_u32(a, b);
+}
+
+// The same pair sums as floats.
+__device__ __forceinline__ float2 e4m3x4_pairsum(uint32_t v) { return h2_to_float2(e4m3x4_pairsum_h(v)); }
 
 // Locate the sequence owning a global block row.
 __device__ __forceinline__ int seq_of_row(const Batch& bt, int row) {
