@@ -45,9 +45,9 @@ KERNEL_SOURCES = ("block_sparse_attention_oam_b200/csrc/stem_bsa.cu", "block_spa
                   "block_sparse_attention_oam_b200/workloads.py")
 MEASURED_TRAFFIC = {
     # (workload, keep, mu, beta): (bytes per launch, sha256 of KERNEL_SOURCES, profile summary)
-    ("qwen3_8b_layer_s128k_fp8", 0.25, 0.7, 0.2): (2.14e9, "0faad37df4b9e65bfff87e4099340736e40601ecb236c8f7db3406492db9a144",
+    ("qwen3_8b_layer_s128k_fp8", 0.25, 0.7, 0.2): (2.14e9, "1a857e2f386235b4a8cd896f9577a462ec053a350e89fcd205bf1ffb1978c8f2",
                                          "profiles/launches_s128k_fp8_keep25.md"),
-    ("qwen3_8b_layer_s64k_bf16", 0.25, 0.7, 0.2): (1.409e9, "0faad37df4b9e65bfff87e4099340736e40601ecb236c8f7db3406492db9a144",
+    ("qwen3_8b_layer_s64k_bf16", 0.25, 0.7, 0.2): (1.413e9, "1a857e2f386235b4a8cd896f9577a462ec053a350e89fcd205bf1ffb1978c8f2",
                                          "profiles/bsa_kernel_bf16_s64k_keep25.md"),
 }
 
@@ -473,20 +473,15 @@ def main():
         S.query_status(ws)
 
     if not args.no_e2e:
-        # end to end through the public API with host buffers: H2D of Q/K/V (pinned),
-        # stem_attention, D2H of the output, every step.
+        # end to end through the C-ABI with host buffers: stem_attention_host copies Q/K/V
+        # (pinned) to the device, runs the path and copies O back, every step; the output
+        # copy overlaps the attention group by group.
         hq, hk, hv = inp.q.pin_memory(), (inp.k_cache if wl.paged else inp.k).pin_memory(), \
             (inp.v_cache if wl.paged else inp.v).pin_memory()
         hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        kd = paged.k_cache if wl.paged else k
-        vd = paged.v_cache if wl.paged else v
 
         def e2e_step():
-            q.copy_(hq, non_blocking=True)
-            kd.copy_(hk, non_blocking=True)
-            vd.copy_(hv, non_blocking=True)
-            S.stem_attention(prob, q, k, v, paged, out=out, ws=ws)
-            hout.copy_(out, non_blocking=True)
+            S.stem_attention_host(prob, hq, hk, hv, q, k, v, paged, out_host=hout, out=out, ws=ws)
 
         for _ in range(2):
             e2e_step()

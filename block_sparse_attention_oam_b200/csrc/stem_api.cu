@@ -323,8 +323,10 @@ stem_status_t do_score(const stem_problem_t* pr, const Batch& bt, const WsLayout
 
 stem_status_t do_bsa(const stem_problem_t* pr, const Batch& bt, const WsLayout& L, const void* q, const void* k,
                      const void* v, const stem_paged_kv_t* pg, const int32_t* row_ptr, const int32_t* col_idx,
-                     void* out, float* lse, void* ws, bool dense, cudaStream_t st) {
+                     void* out, float* lse, void* ws, bool dense, cudaStream_t st, int pair0 = 0, int npairs = 0) {
   BsaArgs a{};
+  a.pair0 = pair0;
+  a.npairs = npairs;
   a.q = q;
   a.k = pg ? pg->k_cache : k;
   a.v = pg ? pg->v_cache : v;
@@ -346,6 +348,54 @@ stem_status_t do_bsa(const stem_problem_t* pr, const Batch& bt, const WsLayout& 
   cudaError_t e = launch_bsa(bt, a, pr->dtype == STEM_DT_FP8_E4M3, pg != nullptr, dense, at<uint32_t>(ws, L.status), st);
   if (e != cudaSuccess) return cuda_fail(e, dense ? "bsa_dense" : "bsa");
   return STEM_OK;
+}
+
+// score -> select into the workspace (the front of stem_attention)
+stem_status_t do_front(const stem_problem_t* pr, const Batch& bt, const WsLayout& L, const void* q, const void* k,
+                       const void* v, const stem_paged_kv_t* pg, void* ws, cudaStream_t st) {
+  stem_status_t s = do_score(pr, bt, L, q, k, v, pg, at<float>(ws, L.scores), ws, st);
+  if (s != STEM_OK) return s;
+  cudaError_t e = launch_select(bt, at<float>(ws, L.scores), pr->num_q_heads, list_group(pr), at<int32_t>(ws, L.row_ptr),
+                                at<int32_t>(ws, L.col_idx), at<uint32_t>(ws, L.status), st);
+  if (e != cudaSuccess) return cuda_fail(e, "select");
+  return STEM_OK;
+}
+
+// the selection kept in the workspace, copied out on request
+stem_status_t copy_selection(const stem_problem_t* pr, const Batch& bt, const WsLayout& L, void* ws,
+                             int32_t* row_ptr_out, int32_t* col_idx_out, cudaStream_t st) {
+  cudaError_t e;
+  if (row_ptr_out != nullptr) {
+    e = cudaMemcpyAsync(row_ptr_out, at<int32_t>(ws, L.row_ptr), (static_cast<size_t>(bt.total_rows) + 1) * 4,
+                        cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "copy row_ptr");
+  }
+  if (col_idx_out != nullptr) {
+    e = cudaMemcpyAsync(col_idx_out, at<int32_t>(ws, L.col_idx), static_cast<size_t>(list_heads(pr)) * bt.nnz_per_head * 4,
+                        cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "copy col_idx");
+  }
+  return STEM_OK;
+}
+
+// One non-blocking stream per device for the output copies of stem_attention_host,
+// created on first use and kept for the life of the process.
+constexpr int kMaxCopyDevices = 64;
+std::mutex g_copy_mu;
+cudaStream_t g_copy_stream[kMaxCopyDevices] = {};
+
+cudaError_t copy_stream_for_current_device(cudaStream_t* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxCopyDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> g(g_copy_mu);
+  if (g_copy_stream[dev] == nullptr) {
+    e = cudaStreamCreateWithFlags(&g_copy_stream[dev], cudaStreamNonBlocking);
+    if (e != cudaSuccess) return e;
+  }
+  *out = g_copy_stream[dev];
+  return cudaSuccess;
 }
 
 stem_status_t check_qkv(const void* q, const void* k, const void* v, const stem_paged_kv_t* pg) {
@@ -481,24 +531,87 @@ stem_status_t stem_attention(const stem_problem_t* prob, const void* q, const vo
   WsLayout L;
   if ((s = check_ws(prob, bt, ws, ws_bytes, &L)) != STEM_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float* scores = at<float>(ws, L.scores);
-  int32_t* rp = at<int32_t>(ws, L.row_ptr);
-  int32_t* ci = at<int32_t>(ws, L.col_idx);
-  if ((s = do_score(prob, bt, L, q, k, v, paged, scores, ws, st)) != STEM_OK) return s;
-  cudaError_t e = launch_select(bt, scores, prob->num_q_heads, list_group(prob), rp, ci, at<uint32_t>(ws, L.status),
-                                st);
-  if (e != cudaSuccess) return cuda_fail(e, "select");
-  if ((s = do_bsa(prob, bt, L, q, k, v, paged, rp, ci, out, lse, ws, false, st)) != STEM_OK) return s;
-  if (row_ptr_out != nullptr) {
-    e = cudaMemcpyAsync(row_ptr_out, rp, (static_cast<size_t>(bt.total_rows) + 1) * 4, cudaMemcpyDeviceToDevice, st);
-    if (e != cudaSuccess) return cuda_fail(e, "copy row_ptr");
+  if ((s = do_front(prob, bt, L, q, k, v, paged, ws, st)) != STEM_OK) return s;
+  if ((s = do_bsa(prob, bt, L, q, k, v, paged, at<int32_t>(ws, L.row_ptr), at<int32_t>(ws, L.col_idx), out, lse, ws,
+                  false, st)) != STEM_OK)
+    return s;
+  return copy_selection(prob, bt, L, ws, row_ptr_out, col_idx_out, st);
+}
+
+stem_status_t stem_attention_host(const stem_problem_t* prob, const void* q_host, const void* k_host,
+                                  const void* v_host, void* q, void* k, void* v, const stem_paged_kv_t* paged,
+                                  void* out_host, void* out, float* lse, int32_t* row_ptr_out, int32_t* col_idx_out,
+                                  int out_groups, void* ws, size_t ws_bytes, void* stream) {
+  stem_status_t s = check_problem(prob);
+  if (s == STEM_OK) s = check_paged(prob, paged);
+  if (s == STEM_OK) s = check_qkv(q, k, v, paged);
+  if (s != STEM_OK) return s;
+  if (q_host == nullptr || k_host == nullptr || v_host == nullptr || out_host == nullptr)
+    return fail(STEM_ERR_INVALID, "q_host, k_host, v_host and out_host must not be NULL");
+  if (out == nullptr || !aligned16(out)) return fail(STEM_ERR_INVALID, "out must be a non-NULL 16-byte aligned pointer");
+  if (out_groups < 0) return fail(STEM_ERR_INVALID, "out_groups %d < 0", out_groups);
+  Batch bt;
+  build_batch(prob, &bt);
+  WsLayout L;
+  if ((s = check_ws(prob, bt, ws, ws_bytes, &L)) != STEM_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t es = prob->dtype == STEM_DT_FP8_E4M3 ? 1 : 2;
+  const size_t d = static_cast<size_t>(prob->head_dim);
+  const size_t T = static_cast<size_t>(bt.total_tokens);
+  const size_t kv_rows = paged ? static_cast<size_t>(paged->num_slots) * STEM_PAGE_SIZE : T;
+  void* kd = paged ? const_cast<void*>(paged->k_cache) : k;
+  void* vd = paged ? const_cast<void*>(paged->v_cache) : v;
+
+  // inputs: host -> device on the caller's stream
+  cudaError_t e = cudaMemcpyAsync(q, q_host, T * prob->num_q_heads * d * es, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(kd, k_host, kv_rows * prob->num_kv_heads * d * es, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(vd, v_host, kv_rows * prob->num_kv_heads * d * es, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return cuda_fail(e, "copy inputs to the device");
+  if ((s = do_front(prob, bt, L, q, k, v, paged, ws, st)) != STEM_OK) return s;
+
+  // attention by groups of head pairs; each group's heads of O go back to the host on
+  // the copy stream while the next groups compute
+  cudaStream_t cs = nullptr;
+  if ((e = copy_stream_for_current_device(&cs)) != cudaSuccess) return cuda_fail(e, "copy stream");
+  const int NP = (prob->num_q_heads + 1) / 2;
+  const int G = out_groups > 0 ? std::min(out_groups, NP) : std::min(8, NP);
+  const size_t row_bytes = static_cast<size_t>(prob->num_q_heads) * d * 2;  // bf16 O
+  cudaEvent_t done = nullptr, copied = nullptr;
+  bool queued = false;  // output copies enqueued on the copy stream
+  for (int g = 0; g < G && s == STEM_OK; ++g) {
+    const int p0 = static_cast<int>(static_cast<long long>(g) * NP / G);
+    const int p1 = static_cast<int>(static_cast<long long>(g + 1) * NP / G);
+    s = do_bsa(prob, bt, L, q, k, v, paged, at<int32_t>(ws, L.row_ptr), at<int32_t>(ws, L.col_idx), out, lse, ws, false,
+               st, p0, p1 - p0);
+    if (s != STEM_OK) break;
+    const int h0 = 2 * p0, h1 = std::min(2 * p1, prob->num_q_heads);
+    e = cudaEventCreateWithFlags(&done, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventRecord(done, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, done, 0);
+    if (done != nullptr) {
+      cudaEventDestroy(done);  // released once the recorded work completes
+      done = nullptr;
+    }
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(static_cast<char*>(out_host) + h0 * d * 2, row_bytes,
+                            static_cast<const char*>(out) + h0 * d * 2, row_bytes, (h1 - h0) * d * 2, T,
+                            cudaMemcpyDeviceToHost, cs);
+    if (e != cudaSuccess) {
+      s = cuda_fail(e, "copy output group to the host");
+      break;
+    }
+    queued = true;
   }
-  if (col_idx_out != nullptr) {
-    e = cudaMemcpyAsync(col_idx_out, ci, static_cast<size_t>(list_heads(prob)) * bt.nnz_per_head * 4,
-                        cudaMemcpyDeviceToDevice, st);
-    if (e != cudaSuccess) return cuda_fail(e, "copy col_idx");
+  if (queued) {
+    // the caller's stream covers every output copy enqueued so far
+    e = cudaEventCreateWithFlags(&copied, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventRecord(copied, cs);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, copied, 0);
+    if (copied != nullptr) cudaEventDestroy(copied);
+    if (e != cudaSuccess && s == STEM_OK) s = cuda_fail(e, "join the copy stream");
   }
-  return STEM_OK;
+  if (s != STEM_OK) return s;
+  return copy_selection(prob, bt, L, ws, row_ptr_out, col_idx_out, st);
 }
 
 stem_status_t stem_query_status(void* ws, void* stream) {

@@ -97,6 +97,8 @@ def lib() -> ctypes.CDLL:
         "bsa_dense_prefill": ([pp, _P, _P, _P, pg, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
         "stem_attention": ([pp, _P, _P, _P, pg, _P, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
         "stem_attention_noalloc": ([pp, _P, _P, _P, pg, _P, _P, _P, _P, _P, _P], ctypes.c_int),
+        "stem_attention_host": ([pp, _P, _P, _P, _P, _P, _P, pg, _P, _P, _P, _P, _P, ctypes.c_int, _P,
+                                 ctypes.c_size_t, _P], ctypes.c_int),
         "stem_query_status": ([_P, _P], ctypes.c_int),
         "stem_reset_status": ([_P, _P], ctypes.c_int),
         "stem_status_string": ([ctypes.c_int], ctypes.c_char_p),
@@ -275,6 +277,28 @@ def capture_attention(prob: Problem, q, k, v, paged: Optional[PagedKV] = None, o
     with torch.cuda.graph(graph):
         stem_attention(prob, q, k, v, paged, out, lse, row_ptr, col_idx, ws)
     return graph, out
+
+
+def stem_attention_host(prob: Problem, q_host, k_host, v_host, q, k, v, paged: Optional[PagedKV] = None,
+                        out_host=None, out=None, lse=None, row_ptr=None, col_idx=None, out_groups: int = 0, ws=None,
+                        stream=None):
+    """The whole path from host tensors: q_host / k_host / v_host (CPU, ideally pinned)
+    are copied into the device tensors q / k / v (a paged cache: into paged.k_cache /
+    paged.v_cache), and O comes back into out_host (CPU bf16 [T, Hq, d]) through the
+    device tensor out, the output copy overlapping the attention group by group.
+    Returns out_host; the copies are asynchronous on `stream` (synchronise before
+    reading it)."""
+    out = _out(prob, q, out)
+    if out_host is None:
+        out_host = torch.empty(tuple(out.shape), dtype=torch.bfloat16, pin_memory=True)
+    for t, name in ((q_host, "q_host"), (k_host, "k_host"), (v_host, "v_host"), (out_host, "out_host")):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous host tensor")
+    ws = workspace(prob, q.device) if ws is None else ws
+    _check(lib().stem_attention_host(prob.c, _ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(q), _ptr(k), _ptr(v),
+                                     _paged(paged), _ptr(out_host), _ptr(out), _ptr(lse), _ptr(row_ptr),
+                                     _ptr(col_idx), int(out_groups), _ptr(ws), ws.numel(), _stream(stream)))
+    return out_host
 
 
 def stem_attention_noalloc(prob: Problem, q, k, v, paged: Optional[PagedKV] = None, out=None, lse=None,

@@ -188,6 +188,32 @@ STEM_API stem_status_t stem_attention(const stem_problem_t* prob, const void* q,
                              int32_t* col_idx_out, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * The whole prefill path from HOST buffers, for end-to-end use (no counterpart in
+ * the pages).  q_host, k_host, v_host: HOST inputs in the layouts of q, k, v (a
+ * paged cache: k_host / v_host hold whole caches of num_slots * page_size rows).
+ * They are copied into the DEVICE buffers q, k, v (for a paged cache into
+ * paged->k_cache / paged->v_cache, which this call overwrites), the path runs as
+ * in stem_attention, and O comes back into out_host (HOST bf16 [T, Hq, d])
+ * through the DEVICE buffer out.  The attention launch is split into out_groups
+ * groups of consecutive head pairs (0: min(8, ceil(Hq / 2)); larger values are
+ * capped at ceil(Hq / 2)); each group's heads of O are copied back on a second
+ * stream while the later groups compute, so most of the output copy overlaps the
+ * attention.  The results equal stem_attention's for any out_groups.  Completion
+ * of the call's work on `stream` includes every copy.  Host buffers should be
+ * page-locked (cudaHostAlloc / cudaHostRegister): pageable ones work but their
+ * copies do not overlap.  lse, row_ptr_out, col_idx_out: DEVICE, as in
+ * stem_attention.  The library keeps one non-blocking copy stream per device
+ * (created on first use) and creates and releases CUDA events per call; it
+ * allocates no device memory.  Errors as stem_attention, plus STEM_ERR_INVALID
+ * for a NULL host pointer or out_groups < 0.
+ */
+STEM_API stem_status_t stem_attention_host(const stem_problem_t* prob, const void* q_host, const void* k_host,
+                                           const void* v_host, void* q, void* k, void* v,
+                                           const stem_paged_kv_t* paged, void* out_host, void* out, float* lse,
+                                           int32_t* row_ptr_out, int32_t* col_idx_out, int out_groups, void* ws,
+                                           size_t ws_bytes, void* stream);
+
+/*
  * stem_attention without a caller workspace, for callers that cannot allocate
  * device memory (a plugin or custom-operator host whose framework owns every
  * byte of the GPU, a serving loop that must not allocate while it runs).  The

@@ -22,7 +22,8 @@ def test_library_exports_every_declared_function(L):
     names = S.header_functions()
     expect = {"stem_query_sizes", "stem_workspace_size", "stem_tpd_plan", "stem_score", "stem_select",
               "bsa_prefill", "bsa_dense_prefill", "stem_attention", "stem_query_status", "stem_reset_status",
-              "stem_status_string", "stem_last_error", "stem_attention_noalloc", "stem_debug_inject"}
+              "stem_status_string", "stem_last_error", "stem_attention_noalloc", "stem_debug_inject",
+              "stem_attention_host"}
     assert expect <= set(names), set(names)
     for n in names:
         assert hasattr(L, n), n
@@ -99,6 +100,23 @@ def test_entry_points_reject_before_launch(L):
     assert st == S.STEM_ERR_INVALID
     assert b"NULL" in L.stem_last_error()
     assert L.stem_status_string(S.STEM_ERR_TIMEOUT) == b"device pipeline wait timed out"
+
+
+def test_host_entry_rejects_before_launch(L):
+    """stem_attention_host refuses NULL host buffers, a negative group count and a
+    short workspace on the host, before any copy or launch."""
+    p = S.Problem([0, 1024], 2, 2, 64, 64)
+    fake = ctypes.c_void_p(0x1000)
+
+    def call(q_host=fake, out_host=fake, groups=0, ws_bytes=1 << 30):
+        return L.stem_attention_host(p.c, q_host, fake, fake, fake, fake, fake, None, out_host, fake, None, None,
+                                     None, groups, fake, ws_bytes, None)
+
+    assert call(q_host=None) == S.STEM_ERR_INVALID
+    assert b"host" in L.stem_last_error()
+    assert call(out_host=None) == S.STEM_ERR_INVALID
+    assert call(groups=-1) == S.STEM_ERR_INVALID
+    assert call(ws_bytes=16) == S.STEM_ERR_WORKSPACE
 
 
 def test_shared_lists_sizes_and_validation(L):
