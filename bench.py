@@ -45,9 +45,9 @@ KERNEL_SOURCES = ("block_sparse_attention_oam_b200/csrc/stem_bsa.cu", "block_spa
                   "block_sparse_attention_oam_b200/workloads.py")
 MEASURED_TRAFFIC = {
     # (workload, keep, mu, beta): (bytes per launch, sha256 of KERNEL_SOURCES, profile summary)
-    ("qwen3_8b_layer_s128k_fp8", 0.25, 0.7, 0.2): (2.14e9, "1a857e2f386235b4a8cd896f9577a462ec053a350e89fcd205bf1ffb1978c8f2",
+    ("qwen3_8b_layer_s128k_fp8", 0.25, 0.7, 0.2): (2.14e9, "0faad37df4b9e65bfff87e4099340736e40601ecb236c8f7db3406492db9a144",
                                          "profiles/launches_s128k_fp8_keep25.md"),
-    ("qwen3_8b_layer_s64k_bf16", 0.25, 0.7, 0.2): (1.413e9, "1a857e2f386235b4a8cd896f9577a462ec053a350e89fcd205bf1ffb1978c8f2",
+    ("qwen3_8b_layer_s64k_bf16", 0.25, 0.7, 0.2): (1.409e9, "0faad37df4b9e65bfff87e4099340736e40601ecb236c8f7db3406492db9a144",
                                          "profiles/bsa_kernel_bf16_s64k_keep25.md"),
 }
 
@@ -474,8 +474,8 @@ def main():
 
     if not args.no_e2e:
         # end to end through the C-ABI with host buffers: stem_attention_host copies Q/K/V
-        # (pinned) to the device, runs the path and copies O back, every step; the output
-        # copy overlaps the attention group by group.
+        # (pinned) to the device, runs the path and copies O back, every step, group of
+        # kv-heads by group, the copies overlapping the work.
         hq, hk, hv = inp.q.pin_memory(), (inp.k_cache if wl.paged else inp.k).pin_memory(), \
             (inp.v_cache if wl.paged else inp.v).pin_memory()
         hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()

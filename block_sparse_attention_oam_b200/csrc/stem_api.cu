@@ -323,10 +323,8 @@ stem_status_t do_score(const stem_problem_t* pr, const Batch& bt, const WsLayout
 
 stem_status_t do_bsa(const stem_problem_t* pr, const Batch& bt, const WsLayout& L, const void* q, const void* k,
                      const void* v, const stem_paged_kv_t* pg, const int32_t* row_ptr, const int32_t* col_idx,
-                     void* out, float* lse, void* ws, bool dense, cudaStream_t st, int pair0 = 0, int npairs = 0) {
+                     void* out, float* lse, void* ws, bool dense, cudaStream_t st) {
   BsaArgs a{};
-  a.pair0 = pair0;
-  a.npairs = npairs;
   a.q = q;
   a.k = pg ? pg->k_cache : k;
   a.v = pg ? pg->v_cache : v;
@@ -378,25 +376,44 @@ stem_status_t copy_selection(const stem_problem_t* pr, const Batch& bt, const Ws
   return STEM_OK;
 }
 
-// One non-blocking stream per device for the output copies of stem_attention_host,
-// created on first use and kept for the life of the process.
+// Two non-blocking streams per device for the copies of stem_attention_host (host to
+// device, device to host), created on first use and kept for the life of the process.
 constexpr int kMaxCopyDevices = 64;
 std::mutex g_copy_mu;
-cudaStream_t g_copy_stream[kMaxCopyDevices] = {};
+cudaStream_t g_copy_streams[kMaxCopyDevices][2] = {};
 
-cudaError_t copy_stream_for_current_device(cudaStream_t* out) {
+cudaError_t copy_streams_for_current_device(cudaStream_t* in, cudaStream_t* out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxCopyDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> g(g_copy_mu);
-  if (g_copy_stream[dev] == nullptr) {
-    e = cudaStreamCreateWithFlags(&g_copy_stream[dev], cudaStreamNonBlocking);
-    if (e != cudaSuccess) return e;
-  }
-  *out = g_copy_stream[dev];
+  for (int i = 0; i < 2; ++i)
+    if (g_copy_streams[dev][i] == nullptr) {
+      e = cudaStreamCreateWithFlags(&g_copy_streams[dev][i], cudaStreamNonBlocking);
+      if (e != cudaSuccess) return e;
+    }
+  *in = g_copy_streams[dev][0];
+  *out = g_copy_streams[dev][1];
   return cudaSuccess;
 }
+
+// CUDA events of one stem_attention_host call, released when the call returns (an event
+// whose recorded work is still pending is freed once that work completes).
+struct CallEvents {
+  std::vector<cudaEvent_t> ev;
+  ~CallEvents() {
+    for (cudaEvent_t e : ev) cudaEventDestroy(e);
+  }
+  cudaError_t record(cudaStream_t on, cudaStream_t waiter) {  // waiter waits for `on`'s work so far
+    cudaEvent_t e = nullptr;
+    cudaError_t r = cudaEventCreateWithFlags(&e, cudaEventDisableTiming);
+    if (r != cudaSuccess) return r;
+    ev.push_back(e);
+    r = cudaEventRecord(e, on);
+    return r == cudaSuccess ? cudaStreamWaitEvent(waiter, e, 0) : r;
+  }
+};
 
 stem_status_t check_qkv(const void* q, const void* k, const void* v, const stem_paged_kv_t* pg) {
   if (q == nullptr || !aligned16(q)) return fail(STEM_ERR_INVALID, "q must be a non-NULL 16-byte aligned pointer");
@@ -554,64 +571,94 @@ stem_status_t stem_attention_host(const stem_problem_t* prob, const void* q_host
   build_batch(prob, &bt);
   WsLayout L;
   if ((s = check_ws(prob, bt, ws, ws_bytes, &L)) != STEM_OK) return s;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  // Groups of kv-heads: the largest divisor of Hkv not above the request (0: 8).  Every
+  // group is a problem of its own (its q-heads, its kv-heads) whose inputs and output
+  // are staged contiguously, group after group, in the device buffers.
+  const int Hq = prob->num_q_heads, Hkv = prob->num_kv_heads;
+  const int want = out_groups > 0 ? out_groups : 8;
+  int G = 1;
+  for (int c = 1; c <= Hkv; ++c)
+    if (Hkv % c == 0 && c <= want) G = c;
+  stem_problem_t sub = *prob;
+  sub.num_q_heads = Hq / G;
+  sub.num_kv_heads = Hkv / G;
+  Batch sbt;
+  build_batch(&sub, &sbt);
+  WsLayout SL;
+  if ((s = check_ws(&sub, sbt, ws, ws_bytes, &SL)) != STEM_OK) return s;
   const size_t es = prob->dtype == STEM_DT_FP8_E4M3 ? 1 : 2;
   const size_t d = static_cast<size_t>(prob->head_dim);
   const size_t T = static_cast<size_t>(bt.total_tokens);
   const size_t kv_rows = paged ? static_cast<size_t>(paged->num_slots) * STEM_PAGE_SIZE : T;
-  void* kd = paged ? const_cast<void*>(paged->k_cache) : k;
-  void* vd = paged ? const_cast<void*>(paged->v_cache) : v;
+  const size_t q_row = static_cast<size_t>(Hq) * d * es, q_grow = static_cast<size_t>(sub.num_q_heads) * d * es;
+  const size_t kv_row = static_cast<size_t>(Hkv) * d * es, kv_grow = static_cast<size_t>(sub.num_kv_heads) * d * es;
+  const size_t o_row = static_cast<size_t>(Hq) * d * 2, o_grow = static_cast<size_t>(sub.num_q_heads) * d * 2;
+  char* qd = static_cast<char*>(q);
+  char* kd = static_cast<char*>(paged ? const_cast<void*>(paged->k_cache) : k);
+  char* vd = static_cast<char*>(paged ? const_cast<void*>(paged->v_cache) : v);
+  char* od = static_cast<char*>(out);
+  const int sub_lists = list_heads(&sub);
 
-  // inputs: host -> device on the caller's stream
-  cudaError_t e = cudaMemcpyAsync(q, q_host, T * prob->num_q_heads * d * es, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(kd, k_host, kv_rows * prob->num_kv_heads * d * es, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(vd, v_host, kv_rows * prob->num_kv_heads * d * es, cudaMemcpyHostToDevice, st);
-  if (e != cudaSuccess) return cuda_fail(e, "copy inputs to the device");
-  if ((s = do_front(prob, bt, L, q, k, v, paged, ws, st)) != STEM_OK) return s;
-
-  // attention by groups of head pairs; each group's heads of O go back to the host on
-  // the copy stream while the next groups compute
-  cudaStream_t cs = nullptr;
-  if ((e = copy_stream_for_current_device(&cs)) != cudaSuccess) return cuda_fail(e, "copy stream");
-  const int NP = (prob->num_q_heads + 1) / 2;
-  const int G = out_groups > 0 ? std::min(out_groups, NP) : std::min(8, NP);
-  const size_t row_bytes = static_cast<size_t>(prob->num_q_heads) * d * 2;  // bf16 O
-  cudaEvent_t done = nullptr, copied = nullptr;
-  bool queued = false;  // output copies enqueued on the copy stream
-  for (int g = 0; g < G && s == STEM_OK; ++g) {
-    const int p0 = static_cast<int>(static_cast<long long>(g) * NP / G);
-    const int p1 = static_cast<int>(static_cast<long long>(g + 1) * NP / G);
-    s = do_bsa(prob, bt, L, q, k, v, paged, at<int32_t>(ws, L.row_ptr), at<int32_t>(ws, L.col_idx), out, lse, ws, false,
-               st, p0, p1 - p0);
-    if (s != STEM_OK) break;
-    const int h0 = 2 * p0, h1 = std::min(2 * p1, prob->num_q_heads);
-    e = cudaEventCreateWithFlags(&done, cudaEventDisableTiming);
-    if (e == cudaSuccess) e = cudaEventRecord(done, st);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, done, 0);
-    if (done != nullptr) {
-      cudaEventDestroy(done);  // released once the recorded work completes
-      done = nullptr;
-    }
+  cudaStream_t st = static_cast<cudaStream_t>(stream), cin = nullptr, cout = nullptr;
+  cudaError_t e = copy_streams_for_current_device(&cin, &cout);
+  if (e != cudaSuccess) return cuda_fail(e, "copy streams");
+  CallEvents ev;
+  // the caller's earlier work on these buffers completes before they are overwritten
+  if ((e = ev.record(st, cin)) != cudaSuccess) return cuda_fail(e, "order the input copies");
+  for (int g = 0; g < G; ++g) {
+    // group g's inputs, host -> device (pitched: its heads out of every token row)
+    e = cudaMemcpy2DAsync(qd + g * T * q_grow, q_grow, static_cast<const char*>(q_host) + g * q_grow, q_row, q_grow, T,
+                          cudaMemcpyHostToDevice, cin);
     if (e == cudaSuccess)
-      e = cudaMemcpy2DAsync(static_cast<char*>(out_host) + h0 * d * 2, row_bytes,
-                            static_cast<const char*>(out) + h0 * d * 2, row_bytes, (h1 - h0) * d * 2, T,
-                            cudaMemcpyDeviceToHost, cs);
+      e = cudaMemcpy2DAsync(kd + g * kv_rows * kv_grow, kv_grow, static_cast<const char*>(k_host) + g * kv_grow,
+                            kv_row, kv_grow, kv_rows, cudaMemcpyHostToDevice, cin);
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(vd + g * kv_rows * kv_grow, kv_grow, static_cast<const char*>(v_host) + g * kv_grow,
+                            kv_row, kv_grow, kv_rows, cudaMemcpyHostToDevice, cin);
+    if (e == cudaSuccess) e = ev.record(cin, st);
     if (e != cudaSuccess) {
-      s = cuda_fail(e, "copy output group to the host");
+      s = cuda_fail(e, "copy inputs to the device");
       break;
     }
-    queued = true;
+    // the path on group g
+    const void* qg = qd + g * T * q_grow;
+    const void* kg = paged ? nullptr : kd + g * kv_rows * kv_grow;
+    const void* vg = paged ? nullptr : vd + g * kv_rows * kv_grow;
+    stem_paged_kv_t pgg{};
+    if (paged) {
+      pgg = *paged;
+      pgg.k_cache = kd + g * kv_rows * kv_grow;
+      pgg.v_cache = vd + g * kv_rows * kv_grow;
+    }
+    const stem_paged_kv_t* pg = paged ? &pgg : nullptr;
+    void* og = od + g * T * o_grow;
+    float* lg = lse ? lse + static_cast<size_t>(g) * sub.num_q_heads * T : nullptr;
+    s = do_front(&sub, sbt, SL, qg, kg, vg, pg, ws, st);
+    if (s == STEM_OK)
+      s = do_bsa(&sub, sbt, SL, qg, kg, vg, pg, at<int32_t>(ws, SL.row_ptr), at<int32_t>(ws, SL.col_idx), og, lg, ws,
+                 false, st);
+    if (s == STEM_OK)
+      s = copy_selection(&sub, sbt, SL, ws, g == 0 ? row_ptr_out : nullptr,
+                         col_idx_out ? col_idx_out + static_cast<size_t>(g) * sub_lists * sbt.nnz_per_head : nullptr,
+                         st);
+    if (s != STEM_OK) break;
+    // group g's output, device -> host, while the next groups compute
+    e = ev.record(st, cout);
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(static_cast<char*>(out_host) + g * o_grow, o_row, og, o_grow, o_grow, T,
+                            cudaMemcpyDeviceToHost, cout);
+    if (e != cudaSuccess) {
+      s = cuda_fail(e, "copy output to the host");
+      break;
+    }
   }
-  if (queued) {
-    // the caller's stream covers every output copy enqueued so far
-    e = cudaEventCreateWithFlags(&copied, cudaEventDisableTiming);
-    if (e == cudaSuccess) e = cudaEventRecord(copied, cs);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, copied, 0);
-    if (copied != nullptr) cudaEventDestroy(copied);
-    if (e != cudaSuccess && s == STEM_OK) s = cuda_fail(e, "join the copy stream");
-  }
+  // the caller's stream covers every copy enqueued (also after an error)
+  cudaError_t j = ev.record(cin, st);
+  if (j == cudaSuccess) j = ev.record(cout, st);
   if (s != STEM_OK) return s;
-  return copy_selection(prob, bt, L, ws, row_ptr_out, col_idx_out, st);
+  if (j != cudaSuccess) return cuda_fail(j, "join the copy streams");
+  return STEM_OK;
 }
 
 stem_status_t stem_query_status(void* ws, void* stream) {

@@ -93,8 +93,7 @@ struct BsaParams {
   void* out;
   float* lse;
   int Hq, Hkv;
-  int pair0, npairs; // the head pairs this launch covers: [pair0, pair0 + npairs)
-  int total_units;   // sum over sequences of N_b * npairs
+  int total_units;   // sum over sequences of N_b * ceil(Hq / 2)
   int groups;        // (sequence, head pair) groups with at least one unit in this launch
   float scale_log2;  // sigma * q_scale * k_scale * log2(e)
   float p_bias;      // log2 of the factor P is scaled by before rounding (FP8: log2 1.75)
@@ -125,7 +124,7 @@ enum : int { kAllRows = 0, kRestRows = 1, kFirstRow = 2 };
 template <int PART>
 __device__ __forceinline__ Unit decode_unit(const BsaParams& p, int u) {
   Unit r{0, 0, 0, false};
-  const int NP = p.npairs;
+  const int NP = (p.Hq + 1) / 2;
   int acc = 0;
   for (int q = 0; q < p.bt.num_seqs; ++q) {
     const int b = p.order[q];
@@ -138,7 +137,7 @@ __device__ __forceinline__ Unit decode_unit(const BsaParams& p, int u) {
       const bool longest_first = ((p.groups - 1 - (q * NP + pair)) & 1) == 0;
       r.b = b;
       r.i = PART == kFirstRow ? 0 : (longest_first ? p.bt.seq[b].nblk - 1 - pos : p.bt.seq[b].nblk - nb + pos);
-      r.h0 = 2 * (p.pair0 + pair);
+      r.h0 = 2 * pair;
       r.two = r.h0 + 1 < p.Hq;
       return r;
     }
@@ -754,7 +753,7 @@ cudaError_t run_part(const BsaParams& prm, bool paged, bool dense, cudaStream_t 
 // first q-block row (where rows have fewer keys than a block) in a small second launch.
 template <int D, int BN, bool FP8>
 cudaError_t run_mode(BsaParams prm, bool paged, bool dense, cudaStream_t st) {
-  const int NP = prm.npairs;
+  const int NP = (prm.Hq + 1) / 2;
   if constexpr (!FP8) {
     long long units = 0;
     for (int b = 0; b < prm.bt.num_seqs; ++b) units += static_cast<long long>(prm.bt.seq[b].nblk) * NP;
@@ -800,10 +799,6 @@ cudaError_t launch_bsa(const Batch& bt, const BsaArgs& a, bool fp8, bool paged, 
   prm.lse = a.lse;
   prm.Hq = a.Hq;
   prm.Hkv = a.Hkv;
-  const int all_pairs = (a.Hq + 1) / 2;
-  prm.pair0 = a.npairs > 0 ? a.pair0 : 0;
-  prm.npairs = a.npairs > 0 ? a.npairs : all_pairs;
-  if (prm.pair0 < 0 || prm.npairs < 1 || prm.pair0 + prm.npairs > all_pairs) return cudaErrorInvalidValue;
   prm.status = status;
   prm.inject = take_injection();
   const float log2e = 1.4426950408889634f;

@@ -412,8 +412,6 @@ struct BsaArgs {
   int Hq, Hkv, head_dim;
   float sigma;
   float q_scale, k_scale, v_scale;
-  int pair0;                // head pairs [pair0, pair0 + npairs) only (q-heads 2p, 2p+1);
-  int npairs;               // npairs 0: every pair
 };
 
 cudaError_t launch_bsa(const Batch& bt, const BsaArgs& a, bool fp8, bool paged, bool dense, uint32_t* status,

@@ -283,11 +283,11 @@ def stem_attention_host(prob: Problem, q_host, k_host, v_host, q, k, v, paged: O
                         out_host=None, out=None, lse=None, row_ptr=None, col_idx=None, out_groups: int = 0, ws=None,
                         stream=None):
     """The whole path from host tensors: q_host / k_host / v_host (CPU, ideally pinned)
-    are copied into the device tensors q / k / v (a paged cache: into paged.k_cache /
-    paged.v_cache), and O comes back into out_host (CPU bf16 [T, Hq, d]) through the
-    device tensor out, the output copy overlapping the attention group by group.
-    Returns out_host; the copies are asynchronous on `stream` (synchronise before
-    reading it)."""
+    go to the device and O comes back into out_host (CPU bf16 [T, Hq, d]), one group of
+    kv-heads at a time, the copies of each group overlapping the work of the others.
+    q / k / v / out (a paged cache: paged.k_cache / paged.v_cache) are device scratch
+    of the full sizes, overwritten with the inputs staged group by group.  Returns
+    out_host; the work is asynchronous on `stream` (synchronise before reading it)."""
     out = _out(prob, q, out)
     if out_host is None:
         out_host = torch.empty(tuple(out.shape), dtype=torch.bfloat16, pin_memory=True)

@@ -191,21 +191,25 @@ STEM_API stem_status_t stem_attention(const stem_problem_t* prob, const void* q,
  * The whole prefill path from HOST buffers, for end-to-end use (no counterpart in
  * the pages).  q_host, k_host, v_host: HOST inputs in the layouts of q, k, v (a
  * paged cache: k_host / v_host hold whole caches of num_slots * page_size rows).
- * They are copied into the DEVICE buffers q, k, v (for a paged cache into
- * paged->k_cache / paged->v_cache, which this call overwrites), the path runs as
- * in stem_attention, and O comes back into out_host (HOST bf16 [T, Hq, d])
- * through the DEVICE buffer out.  The attention launch is split into out_groups
- * groups of consecutive head pairs (0: min(8, ceil(Hq / 2)); larger values are
- * capped at ceil(Hq / 2)); each group's heads of O are copied back on a second
- * stream while the later groups compute, so most of the output copy overlaps the
- * attention.  The results equal stem_attention's for any out_groups.  Completion
- * of the call's work on `stream` includes every copy.  Host buffers should be
- * page-locked (cudaHostAlloc / cudaHostRegister): pageable ones work but their
- * copies do not overlap.  lse, row_ptr_out, col_idx_out: DEVICE, as in
- * stem_attention.  The library keeps one non-blocking copy stream per device
- * (created on first use) and creates and releases CUDA events per call; it
- * allocates no device memory.  Errors as stem_attention, plus STEM_ERR_INVALID
- * for a NULL host pointer or out_groups < 0.
+ * out_host: HOST bf16 [T, Hq, d], receives O.  The kv-heads are split into G
+ * groups, G the largest divisor of Hkv not above out_groups (0: 8); each group
+ * (its kv-heads and their q-heads) is a problem of its own.  Per group, its heads
+ * are copied host -> device, the path runs on them, and their O goes back
+ * device -> host; the input copies, the path and the output copies run on three
+ * streams, so the copies of one group overlap the work of the others.  The results
+ * (out_host, out, lse, the selection) equal stem_attention's for any G.
+ * q, k, v (a paged cache: paged->k_cache, paged->v_cache) and out: DEVICE scratch
+ * of the sizes of the full tensors, which this call overwrites with the inputs and
+ * outputs staged group after group (each group's heads contiguous), not in the
+ * layouts above.  lse: DEVICE [Hq, T] or NULL; row_ptr_out, col_idx_out: DEVICE or
+ * NULL, layouts of stem_select.  Completion of the call's work on `stream` includes
+ * every copy; the device buffers are not overwritten before the caller's earlier
+ * work on `stream` completes.  Host buffers should be page-locked (cudaHostAlloc /
+ * cudaHostRegister): pageable ones work but their copies do not overlap.  The
+ * library keeps two non-blocking copy streams per device (created on first use) and
+ * creates and releases CUDA events per call; it allocates no device memory.
+ * Errors as stem_attention, plus STEM_ERR_INVALID for a NULL host pointer or
+ * out_groups < 0.
  */
 STEM_API stem_status_t stem_attention_host(const stem_problem_t* prob, const void* q_host, const void* k_host,
                                            const void* v_host, void* q, void* k, void* v,

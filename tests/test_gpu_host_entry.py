@@ -1,8 +1,9 @@
-"""stem_attention_host: the whole path from host buffers, with the attention split into
-groups of head pairs whose output copies overlap the later groups.  Every unit is computed
-by the same kernel whatever the grouping, so the output, the log-sum-exp and the selection
-equal stem_attention's bit for bit, for contiguous and paged caches, BF16 and FP8, and any
-number of groups."""
+"""stem_attention_host: the whole path from host buffers, one group of kv-heads at a time,
+each group's copies overlapping the other groups' work.  Every head's arithmetic is
+independent of the other heads, so the output, the log-sum-exp and the selection equal
+stem_attention's bit for bit, for contiguous and paged caches, BF16 and FP8, per-head and
+shared lists, and any number of groups (G = 1, 2, 4 below; an odd number of q-heads per
+group in the ragged case)."""
 import pytest
 import torch
 
@@ -13,7 +14,9 @@ from tests import stem_testlib as T
 pytestmark = pytest.mark.gpu
 
 CASES = {
-    "fp8_gqa_s4096": W.LONG_128K_FP8.with_(name="host_fp8", seqlens=(4096,), num_q_heads=8, num_kv_heads=2, seed=61),
+    "fp8_gqa_s4096": W.LONG_128K_FP8.with_(name="host_fp8", seqlens=(4096,), num_q_heads=8, num_kv_heads=4, seed=61),
+    "bf16_shared_lists": W.QWEN_32K.with_(name="host_shared", seqlens=(2048, 1000), num_q_heads=8, num_kv_heads=2,
+                                         shared_lists=True, seed=64),
     "bf16_ragged_varlen": W.QWEN_32K.with_(name="host_bf16", seqlens=(300, 2112, 1024), num_q_heads=6,
                                           num_kv_heads=2, seed=62),
     "bf16_paged_varlen": W.PAGED_VARLEN.with_(name="host_paged", seqlens=(2048, 640, 4096), num_q_heads=4,
@@ -76,6 +79,11 @@ def test_host_entry_equals_device_entry(name, groups):
     S.query_status(ws)   # synchronises the stream the copies joined
     assert got.data_ptr() == out_host.data_ptr()
     assert torch.equal(out_host.view(torch.int16), ref.view(torch.int16))
-    assert torch.equal(out.cpu().view(torch.int16), ref.view(torch.int16))
+    # the device buffer holds O staged group by group: group g's q-heads contiguous
+    wl = inp.wl
+    G = max(c for c in range(1, wl.num_kv_heads + 1) if wl.num_kv_heads % c == 0 and c <= (groups or 8))
+    hg = wl.num_q_heads // G
+    staged = ref.view(ref.shape[0], G, hg, ref.shape[2]).permute(1, 0, 2, 3).contiguous()
+    assert torch.equal(out.cpu().view(torch.int16).view(G, ref.shape[0], hg, ref.shape[2]), staged.view(torch.int16))
     assert torch.equal(lse.cpu(), ref_lse)
     assert torch.equal(rp.cpu(), ref_rp) and torch.equal(ci.cpu(), ref_ci)
