@@ -119,6 +119,16 @@ def test_host_entry_rejects_before_launch(L):
     assert call(ws_bytes=16) == S.STEM_ERR_WORKSPACE
 
 
+def test_host_entry_binding_checks_host_tensors(L):
+    """The binding refuses device or non-contiguous host tensors before calling the library."""
+    import torch
+    p = S.Problem([0, 256], 2, 2, 64, 64)
+    q = torch.zeros((256, 2, 64), dtype=torch.bfloat16)
+    strided = torch.zeros((256, 2, 128), dtype=torch.bfloat16)[:, :, ::2]
+    with pytest.raises(ValueError, match="k_host"):
+        S.stem_attention_host(p, q, strided, q, q, q, q, out_host=q, out=q, ws=torch.zeros(1 << 20, dtype=torch.uint8))
+
+
 def test_shared_lists_sizes_and_validation(L):
     """One selection per KV group: col_idx has Hkv rows; any other flag value is refused."""
     cu = np.array([0, 1024, 3000])
