@@ -221,7 +221,7 @@ STEM_API stem_status_t stem_attention_host(const stem_problem_t* prob, const voi
  * stem_attention without a caller workspace, for callers that cannot allocate
  * device memory (a plugin or custom-operator host whose framework owns every
  * byte of the GPU, a serving loop that must not allocate while it runs).  The
- * paper has no counterpart: this is a deployment convenience of this library.
+ * pages have no counterpart: this is a deployment convenience of this library.
  * Scratch comes from one fixed 32 MiB array compiled into the library, which
  * every device that loads the library holds until the process exits; a problem
  * whose stem_workspace_size() exceeds it is refused with STEM_ERR_WORKSPACE
