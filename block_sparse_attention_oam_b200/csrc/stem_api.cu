@@ -296,24 +296,27 @@ stem_status_t do_score(const stem_problem_t* pr, const Batch& bt, const WsLayout
   a.scale = fp8 ? pr->q_scale : 1.0f;
   a.mean_out = at<float>(ws, L.qbar);
   a.lognorm_out = nullptr;
-  cudaError_t e = launch_pool(bt, a, pr->head_dim, fp8, false, status, st);
+  a.status = status;
+  cudaError_t e = launch_pool(bt, a, pr->head_dim, fp8, false, st);
   if (e != cudaSuccess) return cuda_fail(e, "pool(Q)");
   PoolArgs kk{};
   kk.x = pg ? pg->k_cache : k;
   kk.block_table = pg ? pg->block_table : nullptr;
   kk.max_pages = pg ? pg->max_pages_per_seq : 0;
+  kk.num_slots = pg ? pg->num_slots : 0;
+  kk.status = status;
   kk.H = pr->num_kv_heads;
   kk.scale = fp8 ? pr->k_scale : 1.0f;
   kk.mean_out = at<float>(ws, L.kbar);
   kk.lognorm_out = nullptr;
-  e = launch_pool(bt, kk, pr->head_dim, fp8, pg != nullptr, status, st);
+  e = launch_pool(bt, kk, pr->head_dim, fp8, pg != nullptr, st);
   if (e != cudaSuccess) return cuda_fail(e, "pool(K)");
   PoolArgs vv = kk;
   vv.x = pg ? pg->v_cache : v;
   vv.scale = fp8 ? pr->v_scale : 1.0f;
   vv.mean_out = nullptr;
   vv.lognorm_out = at<float>(ws, L.lbar);
-  e = launch_pool(bt, vv, pr->head_dim, fp8, pg != nullptr, status, st);
+  e = launch_pool(bt, vv, pr->head_dim, fp8, pg != nullptr, st);
   if (e != cudaSuccess) return cuda_fail(e, "pool(V)");
   e = launch_score(bt, at<float>(ws, L.qbar), at<float>(ws, L.kbar), at<float>(ws, L.lbar), pr->num_q_heads,
                    pr->num_kv_heads, pr->head_dim, sigma_of(pr), pr->beta, scores, st);

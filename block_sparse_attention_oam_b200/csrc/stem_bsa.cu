@@ -288,7 +288,10 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
         for (int s = 0; s < 2; ++s) {
           int myj = jl;
           if (!DENSE) myj = (jl < n && s < ns) ? __ldg(lists[s] + jl) : 0;
-          if (jl < n && s < ns && (myj < 0 || myj > un.i)) {
+          // every entry lies in 0..i and the last one is the diagonal block (the only one
+          // the token-level mask applies to); anything else is reported, and the diagonal
+          // block read in its place
+          if (jl < n && s < ns && (myj < 0 || myj > un.i || (jl == n - 1 && myj != un.i))) {
             atomicOr(p.status, kStatusBounds);
             myj = un.i;
           }

@@ -383,14 +383,15 @@ struct PoolArgs {
   const void* x;            // contiguous [T, H, d] or paged cache [slots, P, H, d]
   const int32_t* block_table;  // paged only
   int max_pages;
+  int num_slots;            // paged only: slots of the cache
+  uint32_t* status;         // device status word (a bad page slot sets the bounds bit)
   int H;
   float scale;              // FP8 dequant scale, 1 for bf16
   float* mean_out;          // [H, R, d]
   float* lognorm_out;       // [H, R] or nullptr
 };
 
-cudaError_t launch_pool(const Batch& bt, const PoolArgs& a, int head_dim, bool fp8, bool paged, uint32_t* status,
-                        cudaStream_t st);
+cudaError_t launch_pool(const Batch& bt, const PoolArgs& a, int head_dim, bool fp8, bool paged, cudaStream_t st);
 cudaError_t launch_score(const Batch& bt, const float* qbar, const float* kbar, const float* lbar, int Hq, int Hkv,
                          int head_dim, float sigma, float beta, float* scores, cudaStream_t st);
 // group = q-heads per list (1: a list per q-head; Hq/Hkv: a list per KV group)

@@ -48,7 +48,10 @@ extern "C" STEM_API stem_status_t stem_attention_noalloc(const stem_problem_t* p
     std::lock_guard<std::mutex> g(g_mu);
     if (g_addr[dev] == nullptr) {
       // host code cannot use g_scratch directly: its name is a host-side shadow,
-      // not a device address.  The device address is looked up once per device.
+      // not a device address.  The device address is looked up once per device and
+      // kept for the life of the process; a device reset (cudaDeviceReset, or a
+      // destroyed and recreated primary context) reloads the module and leaves the
+      // kept address stale, so this entry point must not be used across one.
       void* p = nullptr;
       const cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
       if (e != cudaSuccess || p == nullptr)

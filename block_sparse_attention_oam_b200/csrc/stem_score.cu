@@ -80,7 +80,12 @@ __global__ void __launch_bounds__(kPoolThreads * kPoolGroups) pool_kernel(const 
   auto tok_ptr = [&](int t) -> const uint4* {
     long long rowi;
     if (PAGED) {
+      // a slot outside the cache is reported (bounds error) and slot 0 read instead
       int slot = a.block_table[static_cast<long long>(b) * a.max_pages + t / STEM_PAGE_SIZE];
+      if (slot < 0 || slot >= a.num_slots) {
+        atomicOr(a.status, kStatusBounds);
+        slot = 0;
+      }
       rowi = static_cast<long long>(slot) * STEM_PAGE_SIZE + (t % STEM_PAGE_SIZE);
     } else {
       rowi = static_cast<long long>(s.tok0) + t;
@@ -249,8 +254,7 @@ __global__ void __launch_bounds__(256) score_kernel(const Batch bt, const float*
 
 }  // namespace
 
-cudaError_t launch_pool(const Batch& bt, const PoolArgs& a, int head_dim, bool fp8, bool paged, uint32_t*,
-                        cudaStream_t st) {
+cudaError_t launch_pool(const Batch& bt, const PoolArgs& a, int head_dim, bool fp8, bool paged, cudaStream_t st) {
   if (head_dim == 128) return fp8 ? pool_dispatch_paged<128, true>(bt, a, paged, st)
                                   : pool_dispatch_paged<128, false>(bt, a, paged, st);
   if (head_dim == 64 && !fp8) return pool_dispatch_paged<64, false>(bt, a, paged, st);

@@ -228,7 +228,9 @@ STEM_API stem_status_t stem_attention_host(const stem_problem_t* prob, const voi
  * before anything is launched.  No call allocates or frees device memory.
  * The first call on a device looks up the array's device address (once per
  * device, with that device current), so make that first call before any stream
- * capture.  All calls on a device share the array and it keeps the last call's
+ * capture.  The address is kept for the life of the process: do not call this
+ * entry point again on a device after a device reset (cudaDeviceReset, or its
+ * primary context destroyed and recreated), which moves the array.  All calls on a device share the array and it keeps the last call's
  * contents: calls that overlap on the GPU (other streams, other threads) race
  * and must be serialised by the caller.  The status word is cleared at the start
  * of each call; status_out (DEVICE uint32, or NULL) receives this call's device

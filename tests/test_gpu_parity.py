@@ -257,3 +257,45 @@ def test_corrupt_selection_reports_bounds_error():
     assert e.value.status == S.STEM_ERR_BOUNDS
     S.stem_attention(prob, dev["q"], dev["k"], dev["v"], ws=ws)   # context still healthy
     assert S.query_status(ws) == S.STEM_OK
+
+
+def test_list_not_ending_on_the_diagonal_reports_bounds_error():
+    """The token-level causal mask applies to the last list entry, which must be the
+    diagonal block; a list that ends elsewhere (every entry still within 0..i) is
+    flagged by the kernel and reported as STEM_ERR_BOUNDS."""
+    inp = inputs("gqa_s4096")
+    prob = S.problem_for(inp.wl, inp)
+    dev = T.to_device(inp)
+    lists, (rp, ci) = _oracle_csr(inp)
+    ci = ci.copy()
+    assert ci[1, rp[6] - 1] == 5
+    ci[1, rp[6] - 1] = 4                  # row 5 of head 1 now ends on block 4
+    ws = S.workspace(prob)
+    S.bsa_prefill(prob, dev["q"], dev["k"], dev["v"], torch.from_numpy(rp).cuda(), torch.from_numpy(ci).cuda(), ws=ws)
+    with pytest.raises(S.StemError) as e:
+        S.query_status(ws)
+    assert e.value.status == S.STEM_ERR_BOUNDS
+    S.stem_attention(prob, dev["q"], dev["k"], dev["v"], ws=ws)
+    assert S.query_status(ws) == S.STEM_OK
+
+
+@pytest.mark.parametrize("bad", ["past_end", "negative"])
+def test_corrupt_page_slot_reports_bounds_error_in_scoring(bad):
+    """A block-table entry outside the cache (within a sequence's pages) is caught by
+    the pooling kernel, which reads slot 0 instead and reports STEM_ERR_BOUNDS before
+    the attention kernel runs; the GPU stays usable."""
+    inp = inputs("paged_varlen")
+    prob = S.problem_for(inp.wl, inp)
+    dev = T.to_device(inp)
+    paged = dev["paged"]
+    table = paged.block_table.clone()
+    num_slots = paged.k_cache.shape[0]
+    table[1, 2] = num_slots + 7 if bad == "past_end" else -3   # sequence 1 has 5 pages
+    bad_paged = S.PagedKV(paged.k_cache, paged.v_cache, table)
+    ws = S.workspace(prob)
+    S.stem_score(prob, dev["q"], None, None, bad_paged, ws=ws)
+    with pytest.raises(S.StemError) as e:
+        S.query_status(ws)
+    assert e.value.status == S.STEM_ERR_BOUNDS
+    S.stem_score(prob, dev["q"], None, None, paged, ws=ws)
+    assert S.query_status(ws) == S.STEM_OK
