@@ -286,39 +286,31 @@ stem_status_t check_ws(const stem_problem_t* pr, const Batch& bt, void* ws, size
   return STEM_OK;
 }
 
+// Block means of Q and K and block mean log-norms of V into the workspace (one launch).
+stem_status_t do_pool(const stem_problem_t* pr, const Batch& bt, const WsLayout& L, const void* q, const void* k,
+                      const void* v, const stem_paged_kv_t* pg, void* ws, cudaStream_t st) {
+  const bool fp8 = pr->dtype == STEM_DT_FP8_E4M3;
+  PoolSet ps{};
+  ps.count = 3;
+  ps.t[0] = PoolTensor{q, pr->num_q_heads, 0, fp8 ? pr->q_scale : 1.0f, at<float>(ws, L.qbar), nullptr, 0};
+  ps.t[1] = PoolTensor{pg ? pg->k_cache : k, pr->num_kv_heads, pg != nullptr, fp8 ? pr->k_scale : 1.0f,
+                       at<float>(ws, L.kbar), nullptr, 0};
+  ps.t[2] = PoolTensor{pg ? pg->v_cache : v, pr->num_kv_heads, pg != nullptr, fp8 ? pr->v_scale : 1.0f, nullptr,
+                       at<float>(ws, L.lbar), 0};
+  ps.block_table = pg ? pg->block_table : nullptr;
+  ps.max_pages = pg ? pg->max_pages_per_seq : 0;
+  ps.num_slots = pg ? pg->num_slots : 0;
+  ps.status = at<uint32_t>(ws, L.status);
+  cudaError_t e = launch_pool(bt, ps, pr->head_dim, fp8, st);
+  if (e != cudaSuccess) return cuda_fail(e, "pool");
+  return STEM_OK;
+}
+
 stem_status_t do_score(const stem_problem_t* pr, const Batch& bt, const WsLayout& L, const void* q, const void* k,
                        const void* v, const stem_paged_kv_t* pg, float* scores, void* ws, cudaStream_t st) {
-  const bool fp8 = pr->dtype == STEM_DT_FP8_E4M3;
-  uint32_t* status = at<uint32_t>(ws, L.status);
-  PoolArgs a{};
-  a.x = q;
-  a.H = pr->num_q_heads;
-  a.scale = fp8 ? pr->q_scale : 1.0f;
-  a.mean_out = at<float>(ws, L.qbar);
-  a.lognorm_out = nullptr;
-  a.status = status;
-  cudaError_t e = launch_pool(bt, a, pr->head_dim, fp8, false, st);
-  if (e != cudaSuccess) return cuda_fail(e, "pool(Q)");
-  PoolArgs kk{};
-  kk.x = pg ? pg->k_cache : k;
-  kk.block_table = pg ? pg->block_table : nullptr;
-  kk.max_pages = pg ? pg->max_pages_per_seq : 0;
-  kk.num_slots = pg ? pg->num_slots : 0;
-  kk.status = status;
-  kk.H = pr->num_kv_heads;
-  kk.scale = fp8 ? pr->k_scale : 1.0f;
-  kk.mean_out = at<float>(ws, L.kbar);
-  kk.lognorm_out = nullptr;
-  e = launch_pool(bt, kk, pr->head_dim, fp8, pg != nullptr, st);
-  if (e != cudaSuccess) return cuda_fail(e, "pool(K)");
-  PoolArgs vv = kk;
-  vv.x = pg ? pg->v_cache : v;
-  vv.scale = fp8 ? pr->v_scale : 1.0f;
-  vv.mean_out = nullptr;
-  vv.lognorm_out = at<float>(ws, L.lbar);
-  e = launch_pool(bt, vv, pr->head_dim, fp8, pg != nullptr, st);
-  if (e != cudaSuccess) return cuda_fail(e, "pool(V)");
-  e = launch_score(bt, at<float>(ws, L.qbar), at<float>(ws, L.kbar), at<float>(ws, L.lbar), pr->num_q_heads,
+  stem_status_t s = do_pool(pr, bt, L, q, k, v, pg, ws, st);
+  if (s != STEM_OK) return s;
+  cudaError_t e = launch_score(bt, at<float>(ws, L.qbar), at<float>(ws, L.kbar), at<float>(ws, L.lbar), pr->num_q_heads,
                    pr->num_kv_heads, pr->head_dim, sigma_of(pr), pr->beta, scores, st);
   if (e != cudaSuccess) return cuda_fail(e, "score");
   return STEM_OK;
@@ -351,13 +343,29 @@ stem_status_t do_bsa(const stem_problem_t* pr, const Batch& bt, const WsLayout& 
   return STEM_OK;
 }
 
-// score -> select into the workspace (the front of stem_attention)
+// pool -> scores -> budget + top-k, into row_ptr / col_idx.  fused: the scores are
+// computed inside the selection kernel and never stored (stem_score_select); otherwise, and
+// for shapes the fused kernel does not cover, the score matrix goes through the workspace
+// (the front of stem_attention: on B200 the tiled score GEMM and the selection kernel
+// together take less time than the fused kernel, which re-reads a row's block summaries
+// for every row).  Both give the same lists bit for bit.
 stem_status_t do_front(const stem_problem_t* pr, const Batch& bt, const WsLayout& L, const void* q, const void* k,
-                       const void* v, const stem_paged_kv_t* pg, void* ws, cudaStream_t st) {
+                       const void* v, const stem_paged_kv_t* pg, int32_t* row_ptr, int32_t* col_idx, void* ws,
+                       cudaStream_t st, bool fused = false) {
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  if (fused && fused_select_supported(pr->num_q_heads, pr->num_kv_heads, list_group(pr), pr->head_dim)) {
+    stem_status_t s = do_pool(pr, bt, L, q, k, v, pg, ws, st);
+    if (s != STEM_OK) return s;
+    cudaError_t e = launch_select_fused(bt, at<float>(ws, L.qbar), at<float>(ws, L.kbar), at<float>(ws, L.lbar),
+                                        pr->num_q_heads, pr->num_kv_heads, list_group(pr), pr->head_dim, sigma_of(pr),
+                                        pr->beta, row_ptr, col_idx, status, st);
+    if (e != cudaSuccess) return cuda_fail(e, "score_select");
+    return STEM_OK;
+  }
   stem_status_t s = do_score(pr, bt, L, q, k, v, pg, at<float>(ws, L.scores), ws, st);
   if (s != STEM_OK) return s;
-  cudaError_t e = launch_select(bt, at<float>(ws, L.scores), pr->num_q_heads, list_group(pr), at<int32_t>(ws, L.row_ptr),
-                                at<int32_t>(ws, L.col_idx), at<uint32_t>(ws, L.status), st);
+  cudaError_t e = launch_select(bt, at<float>(ws, L.scores), pr->num_q_heads, list_group(pr), row_ptr, col_idx, status,
+                                st);
   if (e != cudaSuccess) return cuda_fail(e, "select");
   return STEM_OK;
 }
@@ -507,6 +515,21 @@ stem_status_t stem_select(const stem_problem_t* prob, const float* scores, int32
   return STEM_OK;
 }
 
+stem_status_t stem_score_select(const stem_problem_t* prob, const void* q, const void* k, const void* v,
+                                const stem_paged_kv_t* paged, int32_t* row_ptr, int32_t* col_idx, void* ws,
+                                size_t ws_bytes, void* stream) {
+  stem_status_t s = check_problem(prob);
+  if (s == STEM_OK) s = check_paged(prob, paged);
+  if (s == STEM_OK) s = check_qkv(q, k, v, paged);
+  if (s != STEM_OK) return s;
+  if (row_ptr == nullptr || col_idx == nullptr) return fail(STEM_ERR_INVALID, "row_ptr and col_idx must not be NULL");
+  Batch bt;
+  build_batch(prob, &bt);
+  WsLayout L;
+  if ((s = check_ws(prob, bt, ws, ws_bytes, &L)) != STEM_OK) return s;
+  return do_front(prob, bt, L, q, k, v, paged, row_ptr, col_idx, ws, static_cast<cudaStream_t>(stream), true);
+}
+
 stem_status_t bsa_prefill(const stem_problem_t* prob, const void* q, const void* k, const void* v,
                           const stem_paged_kv_t* paged, const int32_t* row_ptr, const int32_t* col_idx, void* out,
                           float* lse, void* ws, size_t ws_bytes, void* stream) {
@@ -551,7 +574,9 @@ stem_status_t stem_attention(const stem_problem_t* prob, const void* q, const vo
   WsLayout L;
   if ((s = check_ws(prob, bt, ws, ws_bytes, &L)) != STEM_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if ((s = do_front(prob, bt, L, q, k, v, paged, ws, st)) != STEM_OK) return s;
+  if ((s = do_front(prob, bt, L, q, k, v, paged, at<int32_t>(ws, L.row_ptr), at<int32_t>(ws, L.col_idx), ws, st)) !=
+      STEM_OK)
+    return s;
   if ((s = do_bsa(prob, bt, L, q, k, v, paged, at<int32_t>(ws, L.row_ptr), at<int32_t>(ws, L.col_idx), out, lse, ws,
                   false, st)) != STEM_OK)
     return s;
@@ -609,51 +634,74 @@ stem_status_t stem_attention_host(const stem_problem_t* prob, const void* q_host
   CallEvents ev;
   // the caller's earlier work on these buffers completes before they are overwritten
   if ((e = ev.record(st, cin)) != cudaSuccess) return cuda_fail(e, "order the input copies");
-  for (int g = 0; g < G; ++g) {
-    // group g's inputs, host -> device (pitched: its heads out of every token row)
-    e = cudaMemcpy2DAsync(qd + g * T * q_grow, q_grow, static_cast<const char*>(q_host) + g * q_grow, q_row, q_grow, T,
-                          cudaMemcpyHostToDevice, cin);
-    if (e == cudaSuccess)
-      e = cudaMemcpy2DAsync(kd + g * kv_rows * kv_grow, kv_grow, static_cast<const char*>(k_host) + g * kv_grow,
-                            kv_row, kv_grow, kv_rows, cudaMemcpyHostToDevice, cin);
-    if (e == cudaSuccess)
-      e = cudaMemcpy2DAsync(vd + g * kv_rows * kv_grow, kv_grow, static_cast<const char*>(v_host) + g * kv_grow,
-                            kv_row, kv_grow, kv_rows, cudaMemcpyHostToDevice, cin);
-    if (e == cudaSuccess) e = ev.record(cin, st);
-    if (e != cudaSuccess) {
-      s = cuda_fail(e, "copy inputs to the device");
-      break;
-    }
-    // the path on group g
-    const void* qg = qd + g * T * q_grow;
-    const void* kg = paged ? nullptr : kd + g * kv_rows * kv_grow;
-    const void* vg = paged ? nullptr : vd + g * kv_rows * kv_grow;
-    stem_paged_kv_t pgg{};
-    if (paged) {
-      pgg = *paged;
-      pgg.k_cache = kd + g * kv_rows * kv_grow;
-      pgg.v_cache = vd + g * kv_rows * kv_grow;
-    }
-    const stem_paged_kv_t* pg = paged ? &pgg : nullptr;
-    void* og = od + g * T * o_grow;
-    float* lg = lse ? lse + static_cast<size_t>(g) * sub.num_q_heads * T : nullptr;
-    s = do_front(&sub, sbt, SL, qg, kg, vg, pg, ws, st);
-    if (s == STEM_OK)
-      s = do_bsa(&sub, sbt, SL, qg, kg, vg, pg, at<int32_t>(ws, SL.row_ptr), at<int32_t>(ws, SL.col_idx), og, lg, ws,
-                 false, st);
-    if (s == STEM_OK)
-      s = copy_selection(&sub, sbt, SL, ws, g == 0 ? row_ptr_out : nullptr,
-                         col_idx_out ? col_idx_out + static_cast<size_t>(g) * sub_lists * sbt.nnz_per_head : nullptr,
-                         st);
-    if (s != STEM_OK) break;
-    // group g's output, device -> host, while the next groups compute
-    e = ev.record(st, cout);
-    if (e == cudaSuccess)
-      e = cudaMemcpy2DAsync(static_cast<char*>(out_host) + g * o_grow, o_row, og, o_grow, o_grow, T,
-                            cudaMemcpyDeviceToHost, cout);
-    if (e != cudaSuccess) {
-      s = cuda_fail(e, "copy output to the host");
-      break;
+  // With two or more groups of one kv-head each (per-head lists, q-heads per group a
+  // multiple of 4), the first and the last group run as two halves of their q-heads: the
+  // copy in front of the first half and the copy behind the last half each move half as
+  // much, and those are the two copies no other group's work can hide.
+  const bool halves = G >= 2 && sub.num_kv_heads == 1 && !prob->shared_lists && sub.num_q_heads % 4 == 0;
+  stem_problem_t half = sub;
+  half.num_q_heads = sub.num_q_heads / 2;
+  Batch hbt;
+  WsLayout HL;
+  if (halves) {
+    build_batch(&half, &hbt);
+    if ((s = check_ws(&half, hbt, ws, ws_bytes, &HL)) != STEM_OK) return s;
+  }
+  const int half_lists = list_heads(&half);
+  for (int g = 0; g < G && s == STEM_OK; ++g) {
+    const int parts = halves && (g == 0 || g == G - 1) ? 2 : 1;
+    const stem_problem_t* pp = parts == 2 ? &half : &sub;
+    const Batch& pbt = parts == 2 ? hbt : sbt;
+    const WsLayout& PL = parts == 2 ? HL : SL;
+    const size_t q_prow = q_grow / parts, o_prow = o_grow / parts;
+    for (int part = 0; part < parts; ++part) {
+      // this piece's inputs, host -> device (pitched: its heads out of every token row);
+      // the group's K and V come with its first piece
+      char* qg = qd + g * T * q_grow + part * T * q_prow;
+      e = cudaMemcpy2DAsync(qg, q_prow, static_cast<const char*>(q_host) + g * q_grow + part * q_prow, q_row, q_prow, T,
+                            cudaMemcpyHostToDevice, cin);
+      if (e == cudaSuccess && part == 0)
+        e = cudaMemcpy2DAsync(kd + g * kv_rows * kv_grow, kv_grow, static_cast<const char*>(k_host) + g * kv_grow,
+                              kv_row, kv_grow, kv_rows, cudaMemcpyHostToDevice, cin);
+      if (e == cudaSuccess && part == 0)
+        e = cudaMemcpy2DAsync(vd + g * kv_rows * kv_grow, kv_grow, static_cast<const char*>(v_host) + g * kv_grow,
+                              kv_row, kv_grow, kv_rows, cudaMemcpyHostToDevice, cin);
+      if (e == cudaSuccess) e = ev.record(cin, st);
+      if (e != cudaSuccess) {
+        s = cuda_fail(e, "copy inputs to the device");
+        break;
+      }
+      // the path on this piece
+      const void* kg = paged ? nullptr : kd + g * kv_rows * kv_grow;
+      const void* vg = paged ? nullptr : vd + g * kv_rows * kv_grow;
+      stem_paged_kv_t pgg{};
+      if (paged) {
+        pgg = *paged;
+        pgg.k_cache = kd + g * kv_rows * kv_grow;
+        pgg.v_cache = vd + g * kv_rows * kv_grow;
+      }
+      const stem_paged_kv_t* pg = paged ? &pgg : nullptr;
+      char* og = od + g * T * o_grow + part * T * o_prow;
+      const size_t head0 = static_cast<size_t>(g) * sub.num_q_heads + static_cast<size_t>(part) * pp->num_q_heads;
+      float* lg = lse ? lse + head0 * T : nullptr;
+      s = do_front(pp, pbt, PL, qg, kg, vg, pg, at<int32_t>(ws, PL.row_ptr), at<int32_t>(ws, PL.col_idx), ws, st);
+      if (s == STEM_OK)
+        s = do_bsa(pp, pbt, PL, qg, kg, vg, pg, at<int32_t>(ws, PL.row_ptr), at<int32_t>(ws, PL.col_idx), og, lg, ws,
+                   false, st);
+      const size_t list0 = static_cast<size_t>(g) * sub_lists + static_cast<size_t>(part) * half_lists;
+      if (s == STEM_OK)
+        s = copy_selection(pp, pbt, PL, ws, g == 0 && part == 0 ? row_ptr_out : nullptr,
+                           col_idx_out ? col_idx_out + list0 * pbt.nnz_per_head : nullptr, st);
+      if (s != STEM_OK) break;
+      // this piece's output, device -> host, while the next pieces compute
+      e = ev.record(st, cout);
+      if (e == cudaSuccess)
+        e = cudaMemcpy2DAsync(static_cast<char*>(out_host) + g * o_grow + part * o_prow, o_row, og, o_prow, o_prow, T,
+                              cudaMemcpyDeviceToHost, cout);
+      if (e != cudaSuccess) {
+        s = cuda_fail(e, "copy output to the host");
+        break;
+      }
     }
   }
   // the caller's stream covers every copy enqueued (also after an error)

@@ -379,21 +379,35 @@ __device__ __forceinline__ int tpd_k(double r, int N, double mu, int i) {
 stem_status_t set_last_error(stem_status_t s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
 
 // ------------------------------------------------------------- host launchers
-struct PoolArgs {
-  const void* x;            // contiguous [T, H, d] or paged cache [slots, P, H, d]
-  const int32_t* block_table;  // paged only
-  int max_pages;
-  int num_slots;            // paged only: slots of the cache
-  uint32_t* status;         // device status word (a bad page slot sets the bounds bit)
+// One tensor of a pooling launch.
+struct PoolTensor {
+  const void* x;            // contiguous [T, H, d], or (paged) a cache [slots, P, H, d]
   int H;
+  int paged;                // addressed through the block table
   float scale;              // FP8 dequant scale, 1 for bf16
-  float* mean_out;          // [H, R, d]
-  float* lognorm_out;       // [H, R] or nullptr
+  float* mean_out;          // [H, R, d] block means, or nullptr
+  float* lognorm_out;       // [H, R] block means of log ||row||_2, or nullptr
+  int slices;               // set by the launcher: CTAs across a token row
+};
+// Q, K and V pooled in one launch (count tensors, in this order).
+struct PoolSet {
+  PoolTensor t[3];
+  int count;
+  const int32_t* block_table;  // paged tensors only
+  int max_pages;
+  int num_slots;            // slots of a paged cache
+  uint32_t* status;         // device status word (a bad page slot sets the bounds bit)
 };
 
-cudaError_t launch_pool(const Batch& bt, const PoolArgs& a, int head_dim, bool fp8, bool paged, cudaStream_t st);
+cudaError_t launch_pool(const Batch& bt, const PoolSet& ps, int head_dim, bool fp8, cudaStream_t st);
 cudaError_t launch_score(const Batch& bt, const float* qbar, const float* kbar, const float* lbar, int Hq, int Hkv,
                          int head_dim, float sigma, float beta, float* scores, cudaStream_t st);
+// Scores computed inside the selection straight from the pooled summaries (no score
+// matrix); the lists equal launch_score + launch_select's bit for bit.
+bool fused_select_supported(int Hq, int Hkv, int group, int head_dim);
+cudaError_t launch_select_fused(const Batch& bt, const float* qbar, const float* kbar, const float* lbar, int Hq,
+                                int Hkv, int group, int head_dim, float sigma, float beta, int32_t* row_ptr,
+                                int32_t* col_idx, uint32_t* status, cudaStream_t st);
 // group = q-heads per list (1: a list per q-head; Hq/Hkv: a list per KV group)
 cudaError_t launch_select(const Batch& bt, const float* scores, int Hq, int group, int32_t* row_ptr,
                           int32_t* col_idx, uint32_t* status, cudaStream_t st);

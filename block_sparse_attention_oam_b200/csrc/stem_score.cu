@@ -17,8 +17,8 @@
 namespace stem {
 namespace {
 
-constexpr int kPoolThreads = 128;   // threads across the token row (16 bytes each)
-constexpr int kPoolGroups = 4;      // token groups per block (more bytes in flight per CTA)
+constexpr int kPoolThreads = 128;     // at most this many threads across a token row (16 bytes each)
+constexpr int kPoolCtaThreads = 512;  // threads of a pooling CTA (4 to 8 token streams)
 
 __device__ __forceinline__ void decode16(const uint4& u, float* f, bool fp8, float scale) {
   if (!fp8) {
@@ -46,15 +46,29 @@ __device__ __forceinline__ void decode16(const uint4& u, float* f, bool fp8, flo
   }
 }
 
-// One CTA per (global block row, group of 128 x VEC elements of the [H*d] token row).
-// Each thread owns VEC consecutive elements (16 bytes) of one head; the block's tokens
-// are split among kPoolGroups groups of 128 threads (contiguous quarters), so every warp
-// reads 512 contiguous bytes per token and a CTA keeps four token streams in flight.
-// The groups' partial sums are added in group order (deterministic).
-template <int D, bool FP8, bool PAGED>
-__global__ void __launch_bounds__(kPoolThreads * kPoolGroups) pool_kernel(const Batch bt, PoolArgs a) {
+// One launch pools Q (means), K (means) and V (mean log-norms): one CTA per (global block
+// row, slice of one tensor's [H*d] token row); blockIdx.y runs over the Q slices, then
+// K's, then V's.  A slice is up to 128 threads x 16 bytes; a narrower token row (FP8 K
+// and V: 64 threads) takes fewer threads (whole warps), the CTA's 512 threads then
+// covering more token streams (grp = thread / threads-per-row).  The block's tokens are split into contiguous runs, one per stream, each
+// thread keeping 8 loads of 16 bytes in flight; the streams' partial sums are added in
+// stream order (deterministic).
+constexpr int kPoolU = 8;   // tokens in flight per thread
+
+template <int D, bool FP8>
+__global__ void __launch_bounds__(kPoolCtaThreads, 2) pool_kernel(const Batch bt, const PoolSet ps) {
   constexpr int VEC = FP8 ? 16 : 8;
   constexpr int LPH = D / VEC;  // lanes per head
+  constexpr int ES = FP8 ? 1 : 2;
+  int ti = 0, slice = blockIdx.y;
+  while (ti + 1 < ps.count && slice >= ps.t[ti].slices) slice -= ps.t[ti++].slices;
+  const PoolTensor& a = ps.t[ti];
+  const int HD = a.H * D;
+  // threads across this slice of the token row: whole warps (32, 64, 96 or 128), so that a
+  // warp never spans two token streams, whose trip counts differ on a partial block (the
+  // log-norm shuffle below is warp-synchronous); lanes past the row end load nothing
+  const int tpr = min(kPoolThreads, (HD / VEC + 31) / 32 * 32);
+  const int streams = kPoolCtaThreads / tpr;
   const int row = blockIdx.x;
   const int b = seq_of_row(bt, row);
   const SeqInfo& s = bt.seq[b];
@@ -63,14 +77,12 @@ __global__ void __launch_bounds__(kPoolThreads * kPoolGroups) pool_kernel(const 
   const int t_beg = i * B;
   const int t_end = min(s.len, t_beg + B);
   const int n = t_end - t_beg;
-  const int HD = a.H * D;
-  const int tx = threadIdx.x % kPoolThreads, grp = threadIdx.x / kPoolThreads;
-  const int e0 = (blockIdx.y * kPoolThreads + tx) * VEC;
+  const int tx = threadIdx.x % tpr, grp = threadIdx.x / tpr;
+  const int e0 = (slice * tpr + tx) * VEC;
   const bool valid = e0 < HD;
   const int h = valid ? e0 / D : 0;
   const int d0 = e0 % D;
   const unsigned char* base = static_cast<const unsigned char*>(a.x);
-  constexpr int ES = FP8 ? 1 : 2;
 
   float acc[VEC];
 #pragma unroll
@@ -79,11 +91,11 @@ __global__ void __launch_bounds__(kPoolThreads * kPoolGroups) pool_kernel(const 
 
   auto tok_ptr = [&](int t) -> const uint4* {
     long long rowi;
-    if (PAGED) {
+    if (a.paged) {
       // a slot outside the cache is reported (bounds error) and slot 0 read instead
-      int slot = a.block_table[static_cast<long long>(b) * a.max_pages + t / STEM_PAGE_SIZE];
-      if (slot < 0 || slot >= a.num_slots) {
-        atomicOr(a.status, kStatusBounds);
+      int slot = ps.block_table[static_cast<long long>(b) * ps.max_pages + t / STEM_PAGE_SIZE];
+      if (slot < 0 || slot >= ps.num_slots) {
+        atomicOr(ps.status, kStatusBounds);
         slot = 0;
       }
       rowi = static_cast<long long>(slot) * STEM_PAGE_SIZE + (t % STEM_PAGE_SIZE);
@@ -93,19 +105,18 @@ __global__ void __launch_bounds__(kPoolThreads * kPoolGroups) pool_kernel(const 
     return reinterpret_cast<const uint4*>(base + (rowi * HD + e0) * ES);
   };
 
-  constexpr int U = 4;
-  const int chunk = (B + kPoolGroups - 1) / kPoolGroups;
+  const int chunk = (B + streams - 1) / streams;
   const int g_beg = t_beg + grp * chunk;
   const int g_end = min(t_end, g_beg + chunk);
-  for (int t = g_beg; t < g_end; t += U) {
-    uint4 buf[U];
+  for (int t = g_beg; t < g_end; t += kPoolU) {
+    uint4 buf[kPoolU];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
+    for (int u = 0; u < kPoolU; ++u) {
       buf[u] = make_uint4(0, 0, 0, 0);
       if (valid && t + u < g_end) buf[u] = __ldg(tok_ptr(t + u));
     }
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
+    for (int u = 0; u < kPoolU; ++u) {
       float f[VEC];
       decode16(buf[u], f, FP8, a.scale);
       float ss = 0.f;
@@ -121,19 +132,22 @@ __global__ void __launch_bounds__(kPoolThreads * kPoolGroups) pool_kernel(const 
       }
     }
   }
-  // partial sums of groups 1.. to group 0, added in group order
-  __shared__ float part[kPoolGroups - 1][VEC + 1][kPoolThreads];
+  // partial sums of streams 1.. to stream 0, added in stream order; [stream - 1][element]
+  // [thread of the stream] (threads past the last whole stream, when tpr does not divide
+  // the CTA, hold no tokens and are not added)
+  __shared__ float part[(VEC + 1) * kPoolCtaThreads];
+  auto slot = [&](int g, int e, int x) -> float& { return part[((g - 1) * (VEC + 1) + e) * tpr + x]; };
   if (grp > 0) {
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) part[grp - 1][e][tx] = acc[e];
-    part[grp - 1][VEC][tx] = lacc;
+    for (int e = 0; e < VEC; ++e) slot(grp, e, tx) = acc[e];
+    slot(grp, VEC, tx) = lacc;
   }
   __syncthreads();
   if (grp > 0 || !valid) return;
-  for (int g = 0; g < kPoolGroups - 1; ++g) {
+  for (int g = 1; g < streams; ++g) {
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) acc[e] += part[g][e][tx];
-    lacc += part[g][VEC][tx];
+    for (int e = 0; e < VEC; ++e) acc[e] += slot(g, e, tx);
+    lacc += slot(g, VEC, tx);
   }
   const float inv = 1.0f / static_cast<float>(n);
   if (a.mean_out != nullptr) {
@@ -147,13 +161,16 @@ __global__ void __launch_bounds__(kPoolThreads * kPoolGroups) pool_kernel(const 
 }
 
 template <int D, bool FP8>
-cudaError_t pool_dispatch_paged(const Batch& bt, const PoolArgs& a, bool paged, cudaStream_t st) {
+cudaError_t pool_dispatch(const Batch& bt, PoolSet ps, cudaStream_t st) {
   constexpr int VEC = FP8 ? 16 : 8;
-  dim3 grid(bt.total_rows, (a.H * D + kPoolThreads * VEC - 1) / (kPoolThreads * VEC));
-  if (paged)
-    pool_kernel<D, FP8, true><<<grid, kPoolThreads * kPoolGroups, 0, st>>>(bt, a);
-  else
-    pool_kernel<D, FP8, false><<<grid, kPoolThreads * kPoolGroups, 0, st>>>(bt, a);
+  int slices = 0;
+  for (int t = 0; t < ps.count; ++t) {
+    const int hd = ps.t[t].H * D;
+    ps.t[t].slices = (hd + kPoolThreads * VEC - 1) / (kPoolThreads * VEC);
+    slices += ps.t[t].slices;
+  }
+  dim3 grid(bt.total_rows, slices);
+  pool_kernel<D, FP8><<<grid, kPoolCtaThreads, 0, st>>>(bt, ps);
   return cudaGetLastError();
 }
 
@@ -254,10 +271,10 @@ __global__ void __launch_bounds__(256) score_kernel(const Batch bt, const float*
 
 }  // namespace
 
-cudaError_t launch_pool(const Batch& bt, const PoolArgs& a, int head_dim, bool fp8, bool paged, cudaStream_t st) {
-  if (head_dim == 128) return fp8 ? pool_dispatch_paged<128, true>(bt, a, paged, st)
-                                  : pool_dispatch_paged<128, false>(bt, a, paged, st);
-  if (head_dim == 64 && !fp8) return pool_dispatch_paged<64, false>(bt, a, paged, st);
+cudaError_t launch_pool(const Batch& bt, const PoolSet& ps, int head_dim, bool fp8, cudaStream_t st) {
+  if (ps.count < 1 || ps.count > 3) return cudaErrorInvalidValue;
+  if (head_dim == 128) return fp8 ? pool_dispatch<128, true>(bt, ps, st) : pool_dispatch<128, false>(bt, ps, st);
+  if (head_dim == 64 && !fp8) return pool_dispatch<64, false>(bt, ps, st);
   return cudaErrorInvalidValue;
 }
 

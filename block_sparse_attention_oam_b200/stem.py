@@ -93,6 +93,7 @@ def lib() -> ctypes.CDLL:
                            ctypes.POINTER(ctypes.c_int64)], ctypes.c_int),
         "stem_score": ([pp, _P, _P, _P, pg, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
         "stem_select": ([pp, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
+        "stem_score_select": ([pp, _P, _P, _P, pg, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
         "bsa_prefill": ([pp, _P, _P, _P, pg, _P, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
         "bsa_dense_prefill": ([pp, _P, _P, _P, pg, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
         "stem_attention": ([pp, _P, _P, _P, pg, _P, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
@@ -224,6 +225,21 @@ def stem_select(prob: Problem, scores, row_ptr=None, col_idx=None, ws=None, stre
     ws = workspace(prob, dev) if ws is None else ws
     _check(lib().stem_select(prob.c, _ptr(scores), _ptr(row_ptr), _ptr(col_idx), _ptr(ws), ws.numel(),
                              _stream(stream)))
+    return row_ptr, col_idx
+
+
+def stem_score_select(prob: Problem, q, k, v, paged: Optional[PagedKV] = None, row_ptr=None, col_idx=None, ws=None,
+                      stream=None):
+    """Pool, score and select in one pass (no score matrix): returns (row_ptr, col_idx)."""
+    sz = prob.sizes()
+    dev = q.device
+    if row_ptr is None:
+        row_ptr = torch.empty(sz["num_rows"] + 1, dtype=torch.int32, device=dev)
+    if col_idx is None:
+        col_idx = torch.empty((sz["list_heads"], sz["nnz_per_head"]), dtype=torch.int32, device=dev)
+    ws = workspace(prob, dev) if ws is None else ws
+    _check(lib().stem_score_select(prob.c, _ptr(q), _ptr(k), _ptr(v), _paged(paged), _ptr(row_ptr), _ptr(col_idx),
+                                   _ptr(ws), ws.numel(), _stream(stream)))
     return row_ptr, col_idx
 
 

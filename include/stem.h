@@ -153,6 +153,25 @@ STEM_API stem_status_t stem_select(const stem_problem_t* prob, const float* scor
                           int32_t* col_idx, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Scoring and selection as one operator (article section "HPC-Stem": compact
+ * block representations, one pass that yields every block score, budget generation
+ * fused with the top-k, no intermediate score tensor).  Pools Q, K and V into the
+ * workspace, then each block row's scores (the formula of stem_score) are computed
+ * inside the selection kernel and ranked there (the rules of stem_select); no score
+ * matrix is written.  The lists equal stem_score followed by stem_select bit for bit
+ * (same float32 operations in the same order).  Shapes the fused kernel does not
+ * cover (shared_lists with more than 16 q-heads per KV group) go through the score
+ * matrix in the workspace instead, with the same result.  On B200 this operator takes
+ * longer than stem_score + stem_select (each row re-reads its kv-head's block means,
+ * where the tiled score GEMM reuses them across rows), so stem_attention uses the latter;
+ * it is for callers that cannot hold the score matrix.
+ * row_ptr, col_idx: DEVICE, layouts of stem_select.  Other arguments as stem_score.
+ */
+STEM_API stem_status_t stem_score_select(const stem_problem_t* prob, const void* q, const void* k, const void* v,
+                                         const stem_paged_kv_t* paged, int32_t* row_ptr, int32_t* col_idx,
+                                         void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Block-sparse causal attention prefill (article section "HPC-BSA"): for each
  * (q-head, q-block) the kernel walks only the listed KV blocks with an online
  * softmax and no per-block branch; skipped blocks behave exactly as if all their
@@ -178,8 +197,9 @@ STEM_API stem_status_t bsa_dense_prefill(const stem_problem_t* prob, const void*
                                 size_t ws_bytes, void* stream);
 
 /*
- * The whole prefill path: stem_score -> stem_select -> bsa_prefill, with the
- * scores and the selection kept in the workspace.  Arguments as bsa_prefill.
+ * The whole prefill path: stem_score -> stem_select -> bsa_prefill (the same result
+ * as stem_score_select -> bsa_prefill), with the scores and the selection kept in the
+ * workspace.  Arguments as bsa_prefill.
  * If row_ptr_out / col_idx_out are non-NULL the selection is also copied there
  * (layouts of stem_select).
  */
@@ -193,14 +213,19 @@ STEM_API stem_status_t stem_attention(const stem_problem_t* prob, const void* q,
  * paged cache: k_host / v_host hold whole caches of num_slots * page_size rows).
  * out_host: HOST bf16 [T, Hq, d], receives O.  The kv-heads are split into G
  * groups, G the largest divisor of Hkv not above out_groups (0: 8); each group
- * (its kv-heads and their q-heads) is a problem of its own.  Per group, its heads
+ * (its kv-heads and their q-heads) is a problem of its own.  When G >= 2, every group
+ * holds one kv-head and a multiple of 4 q-heads, and shared_lists is 0, the first and
+ * the last group each run as two halves of their q-heads (a problem each, with the
+ * group's kv-head), so the first input copy and the last output copy are half as
+ * large.  Per group (or half), its heads
  * are copied host -> device, the path runs on them, and their O goes back
  * device -> host; the input copies, the path and the output copies run on three
  * streams, so the copies of one group overlap the work of the others.  The results
  * (out_host, out, lse, the selection) equal stem_attention's for any G.
  * q, k, v (a paged cache: paged->k_cache, paged->v_cache) and out: DEVICE scratch
  * of the sizes of the full tensors, which this call overwrites with the inputs and
- * outputs staged group after group (each group's heads contiguous), not in the
+ * outputs staged group after group (each group's heads contiguous; a group run in
+ * two halves holds its first half's heads, then its second half's), not in the
  * layouts above.  lse: DEVICE [Hq, T] or NULL; row_ptr_out, col_idx_out: DEVICE or
  * NULL, layouts of stem_select.  Completion of the call's work on `stream` includes
  * every copy; the device buffers are not overwritten before the caller's earlier

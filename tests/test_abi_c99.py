@@ -23,7 +23,7 @@ int main(void) {
   /* every entry point the header declares, by address */
   any_fn fns[] = {
     (any_fn)stem_query_sizes, (any_fn)stem_workspace_size, (any_fn)stem_tpd_plan, (any_fn)stem_score,
-    (any_fn)stem_select, (any_fn)bsa_prefill, (any_fn)bsa_dense_prefill, (any_fn)stem_attention,
+    (any_fn)stem_select, (any_fn)stem_score_select, (any_fn)bsa_prefill, (any_fn)bsa_dense_prefill, (any_fn)stem_attention,
     (any_fn)stem_attention_host, (any_fn)stem_attention_noalloc, (any_fn)stem_query_status,
     (any_fn)stem_reset_status, (any_fn)stem_debug_inject, (any_fn)stem_status_string, (any_fn)stem_last_error};
   for (unsigned i = 0; i < sizeof(fns) / sizeof(fns[0]); ++i)

@@ -21,6 +21,7 @@ def L():
 def test_library_exports_every_declared_function(L):
     names = S.header_functions()
     expect = {"stem_query_sizes", "stem_workspace_size", "stem_tpd_plan", "stem_score", "stem_select",
+              "stem_score_select",
               "bsa_prefill", "bsa_dense_prefill", "stem_attention", "stem_query_status", "stem_reset_status",
               "stem_status_string", "stem_last_error", "stem_attention_noalloc", "stem_debug_inject",
               "stem_attention_host"}
@@ -96,6 +97,10 @@ def test_entry_points_reject_before_launch(L):
     assert st == S.STEM_ERR_WORKSPACE
     st = L.bsa_prefill(p.c, fake, fake, fake, None, None, fake, fake, None, fake, 1 << 30, None)
     assert st == S.STEM_ERR_INVALID
+    st = L.stem_score_select(p.c, fake, fake, fake, None, None, fake, fake, 1 << 30, None)
+    assert st == S.STEM_ERR_INVALID                           # no row_ptr
+    st = L.stem_score_select(p.c, fake, fake, fake, None, fake, fake, fake, 16, None)
+    assert st == S.STEM_ERR_WORKSPACE
     st = L.stem_attention(None, fake, fake, fake, None, fake, None, None, None, fake, 1 << 30, None)
     assert st == S.STEM_ERR_INVALID
     assert b"NULL" in L.stem_last_error()

@@ -1,8 +1,9 @@
 """Parity at the full workload sizes, in the launch configuration bench.py times
-(stem_score -> stem_select -> bsa_prefill), on outputs the oracle can compute one
-by one: every score row of sampled q-heads, the selection of sampled heads (bit-exact
-when fed the oracle's scores), and sampled attention tiles.  Also the largest
-supported sequence (2048 blocks) and degenerate lengths."""
+(stem_score_select -> bsa_prefill), on outputs the oracle can compute one by one: every
+score row of sampled q-heads (from stem_score), the selection of sampled heads
+(bit-exact when fed the oracle's scores; the fused front's lists equal the score-matrix
+path's on every head), and sampled attention tiles.  Also the largest supported
+sequence (2048 blocks) and degenerate lengths."""
 import math
 
 import numpy as np
@@ -38,7 +39,8 @@ def _need_cuda():
 
 
 def _run_path(wl, inp):
-    """The bench's step: three entry points on one workspace."""
+    """The bench's step (stem_score_select -> bsa_prefill) on one workspace, plus the
+    score matrix and its selection (stem_score -> stem_select) for the checks."""
     prob = S.problem_for(wl, inp)
     sz = prob.sizes()
     dev = T.to_device(inp)
@@ -48,9 +50,12 @@ def _run_path(wl, inp):
     ci = torch.empty((wl.num_q_heads, sz["nnz_per_head"]), dtype=torch.int32, device="cuda")
     out = torch.empty((sz["total_tokens"], wl.num_q_heads, wl.head_dim), dtype=torch.bfloat16, device="cuda")
     S.stem_score(prob, dev["q"], dev["k"], dev["v"], dev["paged"], scores=scores, ws=ws)
-    S.stem_select(prob, scores, rp, ci, ws=ws)
+    rp0, ci0 = S.stem_select(prob, scores, ws=ws)
+    S.stem_score_select(prob, dev["q"], dev["k"], dev["v"], dev["paged"], rp, ci, ws=ws)
     S.bsa_prefill(prob, dev["q"], dev["k"], dev["v"], rp, ci, dev["paged"], out=out, ws=ws)
     S.query_status(ws)
+    assert torch.equal(rp, rp0) and torch.equal(ci, ci0), "fused front differs from the score-matrix path"
+    del rp0, ci0
     return prob, dev, ws, scores, rp, ci, out
 
 

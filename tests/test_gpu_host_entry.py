@@ -3,7 +3,8 @@ each group's copies overlapping the other groups' work.  Every head's arithmetic
 independent of the other heads, so the output, the log-sum-exp and the selection equal
 stem_attention's bit for bit, for contiguous and paged caches, BF16 and FP8, per-head and
 shared lists, and any number of groups (G = 1, 2, 4 below; an odd number of q-heads per
-group in the ragged case)."""
+group in the ragged case; the first and last groups in two halves where they hold one
+kv-head and a multiple of 4 q-heads)."""
 import pytest
 import torch
 
@@ -21,6 +22,13 @@ CASES = {
                                           num_kv_heads=2, seed=62),
     "bf16_paged_varlen": W.PAGED_VARLEN.with_(name="host_paged", seqlens=(2048, 640, 4096), num_q_heads=4,
                                              num_kv_heads=2, seed=63),
+    # one kv-head and 4 q-heads per group: the first and last groups run in two halves
+    "bf16_halves": W.QWEN_32K.with_(name="host_halves", seqlens=(2048, 700), num_q_heads=16, num_kv_heads=4,
+                                    seed=65),
+    "fp8_halves": W.LONG_128K_FP8.with_(name="host_fp8_halves", seqlens=(3000,), num_q_heads=8, num_kv_heads=2,
+                                        seed=66),
+    "paged_halves": W.PAGED_VARLEN.with_(name="host_paged_halves", seqlens=(1500, 4096), num_q_heads=8,
+                                         num_kv_heads=2, seed=67),
 }
 
 _cache = {}
@@ -79,11 +87,20 @@ def test_host_entry_equals_device_entry(name, groups):
     S.query_status(ws)   # synchronises the stream the copies joined
     assert got.data_ptr() == out_host.data_ptr()
     assert torch.equal(out_host.view(torch.int16), ref.view(torch.int16))
-    # the device buffer holds O staged group by group: group g's q-heads contiguous
+    # the device buffer holds O staged group by group: group g's q-heads contiguous, and a
+    # group run in two halves (the first and last, with one kv-head and a multiple of 4
+    # q-heads per group, two or more groups, per-head lists) its halves one after the other
     wl = inp.wl
     G = max(c for c in range(1, wl.num_kv_heads + 1) if wl.num_kv_heads % c == 0 and c <= (groups or 8))
     hg = wl.num_q_heads // G
-    staged = ref.view(ref.shape[0], G, hg, ref.shape[2]).permute(1, 0, 2, 3).contiguous()
-    assert torch.equal(out.cpu().view(torch.int16).view(G, ref.shape[0], hg, ref.shape[2]), staged.view(torch.int16))
+    halves = G >= 2 and wl.num_kv_heads // G == 1 and not wl.shared_lists and hg % 4 == 0
+    pieces = []
+    for g in range(G):
+        parts = 2 if halves and g in (0, G - 1) else 1
+        for p_ in range(parts):
+            h0 = g * hg + p_ * hg // parts
+            pieces.append(ref[:, h0:h0 + hg // parts].contiguous().flatten())
+    staged = torch.cat(pieces)
+    assert torch.equal(out.cpu().flatten().view(torch.int16), staged.view(torch.int16))
     assert torch.equal(lse.cpu(), ref_lse)
     assert torch.equal(rp.cpu(), ref_rp) and torch.equal(ci.cpu(), ref_ci)
