@@ -386,7 +386,7 @@ struct PoolTensor {
   int paged;                // addressed through the block table
   float scale;              // FP8 dequant scale, 1 for bf16
   float* mean_out;          // [H, R, d] block means, or nullptr
-  float* lognorm_out;       // [H, R] block means of log ||row||_2, or nullptr
+  float* lognorm_out;       // [H, R] block means of log ||row||_2, or nullptr (exactly one of the two)
   int slices;               // set by the launcher: CTAs across a token row
 };
 // Q, K and V pooled in one launch (count tensors, in this order).

@@ -12,6 +12,8 @@
 #include <cuda_fp16.h>
 #include <float.h>
 
+#include <type_traits>
+
 #include "stem_internal.cuh"
 
 namespace stem {
@@ -20,16 +22,17 @@ namespace {
 constexpr int kPoolThreads = 128;     // at most this many threads across a token row (16 bytes each)
 constexpr int kPoolCtaThreads = 512;  // threads of a pooling CTA (4 to 8 token streams)
 
-__device__ __forceinline__ void decode16(const uint4& u, float* f, bool fp8, float scale) {
+// 16 bytes -> 8 bf16 or 16 e4m3 values as floats (FP8: the codes' values; the per-tensor
+// scale is applied once per block mean or norm, not per element).
+__device__ __forceinline__ void decode16(const uint4& u, float* f, bool fp8) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
   if (!fp8) {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       f[2 * q] = __uint_as_float(w[q] << 16);
       f[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
     }
   } else {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
 #pragma unroll
@@ -37,10 +40,9 @@ __device__ __forceinline__ void decode16(const uint4& u, float* f, bool fp8, flo
         uint16_t pair = static_cast<uint16_t>(w[q] >> (16 * hlf));
         uint32_t h2;
         asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
-        __half2 hv = *reinterpret_cast<__half2*>(&h2);
-        float2 fv = __half22float2(hv);
-        f[4 * q + 2 * hlf] = fv.x * scale;
-        f[4 * q + 2 * hlf + 1] = fv.y * scale;
+        const float2 fv = __half22float2(*reinterpret_cast<__half2*>(&h2));
+        f[4 * q + 2 * hlf] = fv.x;
+        f[4 * q + 2 * hlf + 1] = fv.y;
       }
     }
   }
@@ -50,14 +52,15 @@ __device__ __forceinline__ void decode16(const uint4& u, float* f, bool fp8, flo
 // row, slice of one tensor's [H*d] token row); blockIdx.y runs over the Q slices, then
 // K's, then V's.  A slice is up to 128 threads x 16 bytes; a narrower token row (FP8 K
 // and V: 64 threads) takes fewer threads (whole warps), the CTA's 512 threads then
-// covering more token streams (grp = thread / threads-per-row).  The block's tokens are split into contiguous runs, one per stream, each
-// thread keeping 8 loads of 16 bytes in flight; the streams' partial sums are added in
-// stream order (deterministic).
-constexpr int kPoolU = 8;   // tokens in flight per thread
+// covering more token streams (grp = thread / threads-per-row).  The block's tokens are
+// split into contiguous runs, one per stream, each thread keeping 8 (FP8: 6) loads of 16
+// bytes in flight; the streams' partial sums are added in stream order (deterministic).  A tensor
+// pooled for means only adds; the V pass only forms the per-token norms.
 
 template <int D, bool FP8>
 __global__ void __launch_bounds__(kPoolCtaThreads, 2) pool_kernel(const Batch bt, const PoolSet ps) {
   constexpr int VEC = FP8 ? 16 : 8;
+  constexpr int kPoolU = FP8 ? 6 : 8;  // tokens in flight per thread (FP8: 16 values each)
   constexpr int LPH = D / VEC;  // lanes per head
   constexpr int ES = FP8 ? 1 : 2;
   int ti = 0, slice = blockIdx.y;
@@ -108,30 +111,38 @@ __global__ void __launch_bounds__(kPoolCtaThreads, 2) pool_kernel(const Batch bt
   const int chunk = (B + streams - 1) / streams;
   const int g_beg = t_beg + grp * chunk;
   const int g_end = min(t_end, g_beg + chunk);
-  for (int t = g_beg; t < g_end; t += kPoolU) {
-    uint4 buf[kPoolU];
+  // the token loop, with the per-token norms only for the tensor that needs them (V)
+  auto run = [&](auto norms) {
+    constexpr bool NORMS = decltype(norms)::value;
+    for (int t = g_beg; t < g_end; t += kPoolU) {
+      uint4 buf[kPoolU];
 #pragma unroll
-    for (int u = 0; u < kPoolU; ++u) {
-      buf[u] = make_uint4(0, 0, 0, 0);
-      if (valid && t + u < g_end) buf[u] = __ldg(tok_ptr(t + u));
-    }
-#pragma unroll
-    for (int u = 0; u < kPoolU; ++u) {
-      float f[VEC];
-      decode16(buf[u], f, FP8, a.scale);
-      float ss = 0.f;
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) {
-        acc[e] += f[e];
-        ss = fmaf(f[e], f[e], ss);
+      for (int u = 0; u < kPoolU; ++u) {
+        buf[u] = make_uint4(0, 0, 0, 0);
+        if (valid && t + u < g_end) buf[u] = __ldg(tok_ptr(t + u));
       }
-      if (a.lognorm_out != nullptr) {
 #pragma unroll
-        for (int o = LPH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o, LPH);
-        if (t + u < g_end) lacc += logf(fmaxf(sqrtf(ss), FLT_MIN));
+      for (int u = 0; u < kPoolU; ++u) {
+        float f[VEC];
+        decode16(buf[u], f, FP8);
+        if constexpr (NORMS) {
+          float ss = 0.f;
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) ss = fmaf(f[e], f[e], ss);
+#pragma unroll
+          for (int o = LPH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o, LPH);
+          if (t + u < g_end) lacc += logf(fmaxf(sqrtf(ss) * a.scale, FLT_MIN));
+        } else {
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) acc[e] += f[e];
+        }
       }
     }
-  }
+  };
+  if (a.lognorm_out != nullptr)
+    run(std::true_type{});
+  else
+    run(std::false_type{});
   // partial sums of streams 1.. to stream 0, added in stream order; [stream - 1][element]
   // [thread of the stream] (threads past the last whole stream, when tpr does not divide
   // the CTA, hold no tokens and are not added)
@@ -151,11 +162,12 @@ __global__ void __launch_bounds__(kPoolCtaThreads, 2) pool_kernel(const Batch bt
   }
   const float inv = 1.0f / static_cast<float>(n);
   if (a.mean_out != nullptr) {
+    const float mul = a.scale * inv;  // FP8: the dequantisation scale (1 for bf16)
     float* dst = a.mean_out + (static_cast<long long>(h) * bt.total_rows + row) * D + d0;
 #pragma unroll
     for (int e = 0; e < VEC; e += 4)
       *reinterpret_cast<float4*>(dst + e) =
-          make_float4(acc[e] * inv, acc[e + 1] * inv, acc[e + 2] * inv, acc[e + 3] * inv);
+          make_float4(acc[e] * mul, acc[e + 1] * mul, acc[e + 2] * mul, acc[e + 3] * mul);
   }
   if (a.lognorm_out != nullptr && d0 == 0) a.lognorm_out[static_cast<long long>(h) * bt.total_rows + row] = lacc * inv;
 }
@@ -166,6 +178,8 @@ cudaError_t pool_dispatch(const Batch& bt, PoolSet ps, cudaStream_t st) {
   int slices = 0;
   for (int t = 0; t < ps.count; ++t) {
     const int hd = ps.t[t].H * D;
+    // a tensor is pooled for its means or for its norms, not both
+    if ((ps.t[t].mean_out == nullptr) == (ps.t[t].lognorm_out == nullptr)) return cudaErrorInvalidValue;
     ps.t[t].slices = (hd + kPoolThreads * VEC - 1) / (kPoolThreads * VEC);
     slices += ps.t[t].slices;
   }
