@@ -30,6 +30,10 @@ SMALL = {
                                  seed=15),
     "d128_b64": W.QWEN_32K.with_(name="d128_b64", seqlens=(1536,), num_q_heads=4, num_kv_heads=1, block=64,
                                  seed=16),
+    "fp8_paged_varlen": W.PAGED_VARLEN.with_(name="fp8_paged_varlen", seqlens=(1024, 300, 2112), num_q_heads=8,
+                                             num_kv_heads=2, dtype="fp8_e4m3", seed=17),
+    "fp8_ragged_varlen": W.LONG_128K_FP8.with_(name="fp8_ragged_varlen", seqlens=(300, 1024, 2112, 77), num_q_heads=4,
+                                               num_kv_heads=2, seed=18),
 }
 
 _cache = {}
