@@ -20,6 +20,7 @@ the time of that one layer (strong scaling).
 from __future__ import annotations
 
 import argparse
+import copy
 import hashlib
 import json
 import math
@@ -56,8 +57,8 @@ KERNEL_SOURCES = ("block_sparse_attention_oam_b200/csrc/stem_bsa.cu", "block_spa
                   "block_sparse_attention_oam_b200/workloads.py")
 MEASURED_TRAFFIC = {
     # (workload, keep, mu, beta): (bytes per launch, sha256 of KERNEL_SOURCES)
-    ("qwen3_8b_layer_s128k_fp8", 0.25, 0.7, 0.2): (2.137295616e9, "0c77fe26087effc0ef5ebc7443b7cedbcd4544657dbd15d8725c8cf94478d982"),
-    ("qwen3_8b_layer_s64k_bf16", 0.25, 0.7, 0.2): (1.41113728e9, "0c77fe26087effc0ef5ebc7443b7cedbcd4544657dbd15d8725c8cf94478d982"),
+    ("qwen3_8b_layer_s128k_fp8", 0.25, 0.7, 0.2): (2.135715072e+09, "67443e355e529571d7e23d60a7c498603ad5b19b615c6093af8c701d992d9c05"),
+    ("qwen3_8b_layer_s64k_bf16", 0.25, 0.7, 0.2): (1.409719296e+09, "67443e355e529571d7e23d60a7c498603ad5b19b615c6093af8c701d992d9c05"),
 }
 
 
@@ -263,6 +264,17 @@ class Layer:
         self.ci = torch.empty((sz["list_heads"], sz["nnz_per_head"]), dtype=torch.int32, device="cuda")
         self.out = torch.empty((sz["total_tokens"], self.wl.num_q_heads, self.wl.head_dim), dtype=torch.bfloat16,
                                device="cuda")
+
+    def with_keep(self, keep):
+        """The same inputs and buffers under another keep fraction (a new problem, workspace
+        and selection)."""
+        other = copy.copy(self)
+        other.wl = self.wl.with_(keep=keep)
+        other.prob = S.problem_for(other.wl, self.inp)
+        other.sz = other.prob.sizes()
+        other.ws = S.workspace(other.prob)
+        other.ci = torch.empty((other.sz["list_heads"], other.sz["nnz_per_head"]), dtype=torch.int32, device="cuda")
+        return other
 
     def front(self):
         S.stem_score(self.prob, self.q, self.k, self.v, self.paged, scores=self.scores, ws=self.ws)
@@ -483,10 +495,9 @@ def sweep(wl, steps, warmup):
     rows = []
     dense_ms = None
     point = None
-    base = None
+    base = Layer(wl)
     for keep in W.SWEEP_KEEPS:
-        layer = Layer(wl.with_(keep=keep)) if base is None else _rekeep(base, keep)
-        base = base or layer
+        layer = base.with_keep(keep)
         stream = torch.cuda.current_stream()
         layer.front()
         for _ in range(warmup):
@@ -515,18 +526,6 @@ def sweep(wl, steps, warmup):
     r2 = 1.0 - float(np.sum((y - (slope * x + icpt)) ** 2) / np.sum((y - y.mean()) ** 2))
     return point, {"workload": wl.name, "dense_ms": dense_ms, "steps": steps, "rows": rows,
                    "fit": {"ms_per_tflop": float(slope), "intercept_ms": float(icpt), "r2": r2}}
-
-
-def _rekeep(base, keep):
-    """The same inputs and buffers with another keep fraction (a new problem and selection)."""
-    layer = Layer.__new__(Layer)
-    layer.__dict__.update(base.__dict__)
-    layer.wl = base.wl.with_(keep=keep)
-    layer.prob = S.problem_for(layer.wl, base.inp)
-    layer.sz = layer.prob.sizes()
-    layer.ws = S.workspace(layer.prob)
-    layer.ci = torch.empty((layer.sz["list_heads"], layer.sz["nnz_per_head"]), dtype=torch.int32, device="cuda")
-    return layer
 
 
 def run_sweep_only(args):

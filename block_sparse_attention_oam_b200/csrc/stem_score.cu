@@ -189,7 +189,8 @@ cudaError_t pool_dispatch(const Batch& bt, PoolSet ps, cudaStream_t st) {
 }
 
 // ------------------------------------------------------------------ scores
-// One CTA per (64 x 64 lower-triangular tile of one sequence, q-head).  fp32 SIMT:
+// One CTA per (64 x 64 lower-triangular tile of one sequence, q-head), each thread a 4 x 4
+// block of consecutive rows and columns.  fp32 SIMT:
 // the GEMM is N x N x d per head (about 4 GFLOP at 128K), far below the path's
 // cost, and fp32 keeps the scores within 1e-3 relative of the float64 definition.
 constexpr int kTile = 64;
@@ -199,8 +200,10 @@ __global__ void __launch_bounds__(256) score_kernel(const Batch bt, const float*
                                                     const float* __restrict__ kbar,
                                                     const float* __restrict__ lbar, int Hq, int Hkv, int D,
                                                     float sigma, float beta, float* __restrict__ scores) {
-  __shared__ float Qs[kKc][kTile + 1];
-  __shared__ float Ks[kKc][kTile + 1];
+  // [d][row] with rows padded to 68 floats: a thread's 4 consecutive rows (or columns) are
+  // one 16-byte read
+  __shared__ __align__(16) float Qs[kKc][kTile + 4];
+  __shared__ __align__(16) float Ks[kKc][kTile + 4];
   const int h = blockIdx.y;
   const int kh = h / (Hq / Hkv);
   // decode (sequence, tile row, tile col)
@@ -257,11 +260,9 @@ __global__ void __launch_bounds__(256) score_kernel(const Batch bt, const float*
     __syncthreads();
 #pragma unroll 8
     for (int kk = 0; kk < kKc; ++kk) {
-      float av[4], bv[4];
-#pragma unroll
-      for (int a = 0; a < 4; ++a) av[a] = Qs[kk][ty + 16 * a];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) bv[c] = Ks[kk][tx + 16 * c];
+      const float4 a4 = *reinterpret_cast<const float4*>(&Qs[kk][4 * ty]);
+      const float4 b4 = *reinterpret_cast<const float4*>(&Ks[kk][4 * tx]);
+      const float av[4] = {a4.x, a4.y, a4.z, a4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
       for (int a = 0; a < 4; ++a)
 #pragma unroll
@@ -272,12 +273,12 @@ __global__ void __launch_bounds__(256) score_kernel(const Batch bt, const float*
   const float* lb = lbar + static_cast<long long>(kh) * R + s.row0;
 #pragma unroll
   for (int a = 0; a < 4; ++a) {
-    const int i = i0 + ty + 16 * a;
+    const int i = i0 + 4 * ty + a;
     if (i >= N) continue;
     const long long roff = static_cast<long long>(i) * (i + 1) / 2;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      const int j = j0 + tx + 16 * c;
+      const int j = j0 + 4 * tx + c;
       if (j <= i) out[roff + j] = fmaf(sigma, acc[a][c], beta * lb[j]);
     }
   }

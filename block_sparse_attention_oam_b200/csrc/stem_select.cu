@@ -94,8 +94,8 @@ __device__ __forceinline__ bool trivial_list(int i, int k_i, int32_t* out, int l
 
 // One warp ranks keys[1..i-1] (order-preserving score keys) and writes the list: block 0,
 // the `need` best candidates under (key descending, index ascending), block i.  A
-// most-significant-digit-first radix select (4 passes of 8 bits, histogram in shared
-// memory) finds the need-th largest key, then a ballot compaction walks the candidates in
+// most-significant-digit-first radix select (8-bit digits below the bits all candidates
+// share, histogram in shared memory) finds the need-th largest key, then a ballot compaction walks the candidates in
 // ascending block order, taking every key above it and the lowest-index keys equal to it.
 // (Measured slower for the 128K layer: a one-bit-at-a-time select with warp-reduced
 // counts and no atomics, 0.22 ms, and one atomic per distinct digit of a warp's keys
@@ -103,14 +103,30 @@ __device__ __forceinline__ bool trivial_list(int i, int k_i, int32_t* out, int l
 __device__ __forceinline__ void select_warp(const uint32_t* keys, uint32_t* hist, int i, int need, int32_t* out,
                                             int lane) {
   const unsigned full = 0xffffffffu;
-  uint32_t prefix = 0, pmask = 0;
+  // the bits every candidate key shares are fixed at once (a row's scores share their
+  // sign and leading exponent bits); the 8-bit digits start below them, so the first pass
+  // spreads the keys over many bins instead of piling them into one or two
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  for (int j = 1 + lane; j < i; j += 32) {
+    const uint32_t u = keys[j];
+    kmin = min(kmin, u);
+    kmax = max(kmax, u);
+  }
+  kmin = __reduce_min_sync(full, kmin);
+  kmax = __reduce_max_sync(full, kmax);
+  const uint32_t diff = kmin ^ kmax;
+  const int top = diff != 0u ? 31 - __clz(diff) : -1;            // highest bit the keys differ in
+  uint32_t pmask = top >= 0 ? ~((2u << top) - 1u) : 0xFFFFFFFFu;  // 2u << 31 wraps to 0: no common bits
+  uint32_t prefix = kmin & pmask;
   int rem = need;
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  for (int hi = top; hi >= 0; hi -= 8) {
+    const int shift = hi >= 7 ? hi - 7 : 0;
+    const uint32_t dmask = (2u << (hi - shift)) - 1u;              // digit of hi - shift + 1 <= 8 bits
     for (int q = lane; q < 256; q += 32) hist[q] = 0;
     __syncwarp();
     for (int j = 1 + lane; j < i; j += 32) {
       const uint32_t u = keys[j];
-      if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+      if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & dmask], 1u);
     }
     __syncwarp();
     int c[8];
@@ -142,7 +158,7 @@ __device__ __forceinline__ void select_warp(const uint32_t* keys, uint32_t* hist
     const int digit = __shfl_sync(full, found, src);
     rem -= __shfl_sync(full, found_above, src);
     prefix |= static_cast<uint32_t>(digit) << shift;
-    pmask |= 0xFFu << shift;
+    pmask |= dmask << shift;
     __syncwarp();
   }
   // prefix = key of the need-th best candidate; rem = how many keys equal to it to take

@@ -16,6 +16,24 @@ SCORE_ATOL = 1e-5
 SCORE_GAP = 1e-3     # end-to-end lists may differ only where the score gap is below this
 
 
+def bf16_half_ulp(x):
+    """Half a bf16 unit in the last place at |x| (8 significand bits): the rounding error the
+    bf16 output format adds on its own to an exact result."""
+    a = np.maximum(np.abs(np.asarray(x, dtype=np.float64)), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 8)
+
+
+def out_bound(ref, base):
+    """Element-wise bound for a bf16 output against the float64 oracle: `base` for the
+    arithmetic (bf16 or FP8 operands, float32 accumulation) plus the output's own rounding."""
+    return base + bf16_half_ulp(ref)
+
+
+def out_excess(got, ref, base):
+    """Largest (|got - ref| - bound); <= 0 means every element is within its bound."""
+    return float((np.abs(got - ref) - out_bound(ref, base)).max())
+
+
 def to_device(inp: W.Inputs):
     d = dict(q=inp.q.cuda(), k=inp.k.cuda(), v=inp.v.cuda(), paged=None)
     if inp.wl.paged:

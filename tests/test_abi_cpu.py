@@ -87,6 +87,15 @@ def test_fp8_shape_limits_and_bad_seqlens(L):
     assert e.value.status == S.STEM_ERR_UNSUPPORTED
 
 
+def test_batch_size_limit(L):
+    """STEM_MAX_SEQS sequences are accepted, one more is refused on the host."""
+    cu = [64 * b for b in range(65)]
+    assert S.Problem(cu, 4, 2, 128, 64).sizes()["num_rows"] == 64
+    with pytest.raises(S.StemError) as e:
+        S.Problem(cu + [cu[-1] + 64], 4, 2, 128, 64).sizes()
+    assert e.value.status == S.STEM_ERR_INVALID
+
+
 def test_entry_points_reject_before_launch(L):
     """Null pointers and a short workspace are refused on the host (no CUDA call)."""
     p = S.Problem([0, 1024], 2, 2, 64, 64)

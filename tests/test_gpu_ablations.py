@@ -126,5 +126,5 @@ def test_ablation_end_to_end(name, ablation):
             k = T.oracle_dequant(inp, "k", t0, t1, [h // g])
             v = T.oracle_dequant(inp, "v", t0, t1, [h // g])
             ref, _ = O.attend(q, k, v, [gl], wl.block, wl.softmax_scale)
-            assert np.abs(out[t0:t1, h] - ref[:, 0]).max() <= tol, (name, ablation, b, h)
+            assert T.out_excess(out[t0:t1, h], ref[:, 0], tol) <= 0, (name, ablation, b, h)
         row0 += N

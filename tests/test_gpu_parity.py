@@ -2,7 +2,8 @@
 float64 oracle on the same seeded inputs.
 
 Bars: scores within 1e-3 relative; selection bit-exact when fed the oracle's
-scores; BF16 outputs within 2e-2 max-abs (FP8 6e-2) of the oracle; end-to-end
+scores; BF16 outputs within 2e-2 (FP8 6e-2) plus half a bf16 ulp of the oracle's
+value (the output format's own rounding) element by element; end-to-end
 lists differ from the oracle's only where the score gap is below 1e-3."""
 import math
 
@@ -34,6 +35,15 @@ SMALL = {
                                              num_kv_heads=2, dtype="fp8_e4m3", seed=17),
     "fp8_ragged_varlen": W.LONG_128K_FP8.with_(name="fp8_ragged_varlen", seqlens=(300, 1024, 2112, 77), num_q_heads=4,
                                                num_kv_heads=2, seed=18),
+    # an odd number of q-heads: the last head pair of every row has one head
+    "odd_heads": W.QWEN_32K.with_(name="odd_heads", seqlens=(1500, 400), num_q_heads=3, num_kv_heads=1, seed=19),
+    # the most sequences a batch may hold (STEM_MAX_SEQS), of seeded lengths 1..299
+    "max_seqs_64": W.QWEN_32K.with_(name="max_seqs_64", seqlens=(
+        177, 126, 107, 277, 114, 82, 263, 18, 133, 93, 9, 215, 298, 234, 97, 162, 254, 94, 128, 274,
+        59, 278, 203, 131, 236, 123, 108, 184, 276, 214, 200, 186, 251, 130, 222, 133, 181, 194,
+        110, 275, 73, 15, 223, 27, 163, 228, 51, 138, 173, 233, 150, 162, 166, 139, 10, 286, 250,
+        111, 110, 194, 267, 163, 82, 34),
+                                    num_q_heads=4, num_kv_heads=2, seed=20),
 }
 
 _cache = {}
@@ -146,7 +156,7 @@ def test_bsa_matches_oracle_attention(name):
     out = out.float().cpu().numpy()
     lse = lse.cpu().numpy()
     tol = T.FP8_TOL if wl.dtype == "fp8_e4m3" else T.BF16_TOL
-    worst = 0.0
+    worst = -np.inf
     for b, (t0, t1) in enumerate(T.seq_slices(inp)):
         N = _seq_blocks(wl)[b]
         for h in range(wl.num_q_heads):
@@ -155,9 +165,9 @@ def test_bsa_matches_oracle_attention(name):
             k = T.oracle_dequant(inp, "k", t0, t1, [h // g])
             v = T.oracle_dequant(inp, "v", t0, t1, [h // g])
             ref, ref_lse = O.attend(q, k, v, [lists[b][h]], wl.block, wl.softmax_scale)
-            err = np.abs(out[t0:t1, h, :] - ref[:, 0, :]).max()
+            err = T.out_excess(out[t0:t1, h, :], ref[:, 0, :], tol)
             worst = max(worst, err)
-            assert err <= tol, (b, h, err)
+            assert err <= 0, (b, h, err)
             assert np.abs(lse[h, t0:t1] - ref_lse[0]).max() <= 2e-3 * max(1.0, np.abs(ref_lse).max())
     assert np.isfinite(out).all()
 
@@ -187,7 +197,7 @@ def test_dense_kernel_equals_keep_one_selection_and_oracle(name):
         v = torch.from_numpy(np.repeat(T.oracle_dequant(inp, "v", t0, t1), g, axis=1)).permute(1, 0, 2)[None]
         ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True, scale=wl.softmax_scale)
         ref = ref[0].permute(1, 0, 2).numpy()
-        assert np.abs(out[t0:t1] - ref).max() <= tol
+        assert T.out_excess(out[t0:t1], ref, tol) <= 0
 
 
 def _check_lists_within_gap(gpu_lists, ora_lists, scores):
@@ -230,7 +240,7 @@ def test_stem_attention_end_to_end(name):
             k = T.oracle_dequant(inp, "k", t0, t1, [h // g])
             v = T.oracle_dequant(inp, "v", t0, t1, [h // g])
             ref, _ = O.attend(q, k, v, [[list(map(int, x)) for x in gl]], wl.block, wl.softmax_scale)
-            assert np.abs(out[t0:t1, h] - ref[:, 0]).max() <= tol
+            assert T.out_excess(out[t0:t1, h], ref[:, 0], tol) <= 0
         row0 += N
 
 
