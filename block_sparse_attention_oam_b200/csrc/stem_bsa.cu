@@ -25,8 +25,9 @@
 //               block (always the last list entry); O rescaled lazily (only when the
 //               running max grows by more than 2^8) — no wait is needed for that, since
 //               S_j is issued after P V_{j-1} and the tensor core runs in order; O
-//               normalised by the sum of the rounded P weights the product used; then the
-//               epilogue (O / l -> bf16, log-sum-exp).
+//               normalised by the sum of the P weights (BF16: as rounded for the product;
+//               FP8: unrounded, except on a sequence's first row); then the epilogue
+//               (O / l -> bf16, log-sum-exp).
 // Every wait is bounded (2 s); on expiry the CTA raises an abort flag, records
 // STEM_ERR_TIMEOUT in the status word, drains its tensor-core work, waits (bounded)
 // for its copies and releases its TMEM before exiting.
@@ -491,8 +492,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
       const int n = unit_len<DENSE>(p, un);
       if (n == 0 || (slot == 1 && !un.two)) continue;
       const int h = un.h0 + slot;
-      // running max; sums of the rounded P the product uses (normalise O) and, for FP8,
-      // of the unrounded P (log-sum-exp)
+      // running max; sums of P that normalise O and, for the FP8 first row, of the
+      // unrounded P (log-sum-exp)
       float m_run = -INFINITY;
       float2 l2 = make_float2(0.f, 0.f), lt2 = make_float2(0.f, 0.f);
       for (int jj = 0; jj < n; ++jj, ++gb) {
@@ -543,10 +544,12 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
               sq[u2 % 4] = add2(sq[u2 % 4], make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
             }
           } else {
-            // sums of the rounded P: the e4m3 weights (exact in f16) go into two f16x2
+            // Rows 1..: O is normalised by the float32 sum of the unrounded weights (the
+            // same sum the log-sum-exp takes).  First row (two-term P): by the sum of the
+            // rounded terms, the e4m3 weights (exact in f16) going into two f16x2
             // accumulators, one weight per lane and quad (relative rounding 2^-11 per
-            // addition), which are added in f32 every 16 quads — fewer conversions and
-            // shorter dependency chains on the exponential phase than a per-quad f32 sum
+            // addition), added in f32 every 16 quads.
+            constexpr bool kRoundedSum = PART == kFirstRow;
             uint32_t hs[2] = {0u, 0u};
 #pragma unroll
             for (int u4 = 0; u4 < BN / 4; ++u4) {
@@ -556,14 +559,16 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
               const float2 e1 = make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
               const uint32_t w = __byte_perm(pack_e4m3x2(e0.x, e0.y), pack_e4m3x2(e1.x, e1.y), 0x5410);
               sr[u4] = w;
-              {
+              if constexpr (!kRoundedSum) {
+                sq[u4 % 4] = add2(sq[u4 % 4], add2(e0, e1));
+              } else {
                 uint32_t a, b;
                 asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(a) : "h"(static_cast<uint16_t>(w & 0xFFFFu)));
                 asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(b) : "h"(static_cast<uint16_t>(w >> 16)));
                 hs[0] = hadd2_u32(hs[0], a);
                 hs[1] = hadd2_u32(hs[1], b);
               }
-              if (u4 % 16 == 15) {
+              if (kRoundedSum && u4 % 16 == 15) {
                 sq[(u4 / 16) % 4] = add2(sq[(u4 / 16) % 4], add2(h2_to_float2(hs[0]), h2_to_float2(hs[1])));
                 hs[0] = 0u;
                 hs[1] = 0u;
@@ -572,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
             }
           }
         };
-        // LSEX (FP8 with a log-sum-exp requested): also the sums of the unrounded P
+        // LSEX (FP8 first row with a log-sum-exp requested): also the sums of the unrounded P
         exps(std::bool_constant<LSEX>{});
         if constexpr (FP8 && PART == kFirstRow) {
           {
@@ -668,7 +673,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
         }
       }
       if (p.lse != nullptr && r < rows_valid) {
-        const float lt = LSEX ? (lt2.x + lt2.y) / p.p_scale : l;
+        // the sum of the unrounded weights (BF16: of the rounded ones; the factor is 1)
+        const float lt = (LSEX ? lt2.x + lt2.y : l) / p.p_scale;
         p.lse[static_cast<long long>(h) * p.bt.total_tokens + tok] = (m_run + __log2f(lt)) * 0.69314718055994531f;
       }
       tc_fence_before();
@@ -729,11 +735,11 @@ cudaError_t run_k(const BsaParams& prm, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-// FP8 with a log-sum-exp requested keeps the unrounded P sums as well (its own kernel, so
-// the default one carries none of that work)
+// The FP8 first-row launch with a log-sum-exp requested keeps the unrounded P sums beside
+// the rounded ones it normalises by (its own kernel, so the default one carries none of it)
 template <int D, int BN, bool FP8, bool PAGED, bool DENSE, int PART, bool SHKV = false>
 cudaError_t run(const BsaParams& prm, cudaStream_t st) {
-  if constexpr (FP8) {
+  if constexpr (FP8 && PART == kFirstRow) {
     if (prm.lse != nullptr) return run_k<D, BN, FP8, PAGED, DENSE, PART, SHKV, true>(prm, st);
   }
   return run_k<D, BN, FP8, PAGED, DENSE, PART, SHKV, false>(prm, st);
@@ -809,7 +815,7 @@ cudaError_t launch_bsa(const Batch& bt, const BsaArgs& a, bool fp8, bool paged, 
   // FP8: P <= 2^8 after the lazy max update; 448 / 256 keeps it inside e4m3's range.
   prm.p_scale = fp8 ? 1.75f : 1.0f;
   prm.p_bias = fp8 ? 0.80735492205760410f : 0.0f;  // log2(1.75)
-  // l is accumulated from the scaled, rounded P, so the V scale is all that remains
+  // l is accumulated from the scaled P, so the V scale is all that remains
   prm.out_scale = fp8 ? a.v_scale : 1.0f;
   // sequences by decreasing block count (longest rows first)
   int ord[STEM_MAX_SEQS];
