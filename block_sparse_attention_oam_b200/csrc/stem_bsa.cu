@@ -147,6 +147,20 @@ __device__ __forceinline__ Unit decode_unit(const BsaParams& p, int u) {
   return r;
 }
 
+// The CTAs take the units round robin (CTA c: c, c + gridDim, ...).  With an odd number
+// of groups the last one has no partner running the other way (a single head pair:
+// nothing cancels, and CTA 0 gets the longest row of every round, 12 % above the mean at
+// 128K); those launches (the SNAKE kernels) deal every window of 2 x gridDim units
+// forwards and back instead, so that each CTA pairs a longer row with a shorter one
+// (1.6 % at 128K; three pairs 4 % -> 1.3 %).  snake_unit: the CTA's k-th unit, or
+// total_units when it has none left.
+__device__ __forceinline__ int snake_unit(const BsaParams& p, int k) {
+  const int g = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x), base = (k >> 1) * 2 * g;
+  if ((k & 1) == 0) return min(base + c, p.total_units);
+  const int len = min(2 * g, p.total_units - base);
+  return c < len - g ? base + len - 1 - c : p.total_units;
+}
+
 // Warp-uniform bounded wait on an mbarrier phase.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           uint32_t* status) {
@@ -184,7 +198,7 @@ __device__ __forceinline__ const int32_t* head_list(const BsaParams& p, const Un
   return p.col_idx + static_cast<long long>(h / p.list_group) * p.bt.nnz_per_head + p.row_ptr[row];
 }
 
-template <int D, int BN, bool FP8, bool PAGED, bool DENSE, int PART, bool SHKV, bool LSEX>
+template <int D, int BN, bool FP8, bool PAGED, bool DENSE, int PART, bool SHKV, bool LSEX, bool SNAKE>
 __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant__ BsaParams p) {
   using C = Cfg<D, BN, FP8>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -258,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
     }
     uint32_t itk[2] = {0, 0}, itv[2] = {0, 0}, tq = 0;
     bool alive = true;
-    for (int u = blockIdx.x; u < p.total_units && alive; u += gridDim.x) {
+    for (int k = 0, u = blockIdx.x; u < p.total_units && alive; u = SNAKE ? snake_unit(p, ++k) : u + gridDim.x) {
       const Unit un = decode_unit<PART>(p, u);
       const int n = unit_len<DENSE>(p, un);
       if (n == 0) {
@@ -397,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
         ++itk[s];
         return true;
       };
-      for (int u = blockIdx.x; u < p.total_units && alive; u += gridDim.x) {
+      for (int k = 0, u = blockIdx.x; u < p.total_units && alive; u = SNAKE ? snake_unit(p, ++k) : u + gridDim.x) {
         const Unit un = decode_unit<PART>(p, u);
         const int n = unit_len<DENSE>(p, un);
         if (n == 0) continue;
@@ -487,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_kernel(const __grid_constant_
     const float sl2 = p.scale_log2;
     uint32_t gb = 0, ot = 0;                         // blocks and units processed by this slot
     bool alive = true;
-    for (int u = blockIdx.x; u < p.total_units && alive; u += gridDim.x) {
+    for (int k = 0, u = blockIdx.x; u < p.total_units && alive; u = SNAKE ? snake_unit(p, ++k) : u + gridDim.x) {
       const Unit un = decode_unit<PART>(p, u);
       const int n = unit_len<DENSE>(p, un);
       if (n == 0 || (slot == 1 && !un.two)) continue;
@@ -720,11 +734,11 @@ bool make_map(CUtensorMap* m, const void* ptr, bool fp8, int d, int H, long long
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int BN, bool FP8, bool PAGED, bool DENSE, int PART, bool SHKV, bool LSEX>
+template <int D, int BN, bool FP8, bool PAGED, bool DENSE, int PART, bool SHKV, bool LSEX, bool SNAKE>
 cudaError_t run_k(const BsaParams& prm, cudaStream_t st) {
   using C = Cfg<D, BN, FP8>;
-  auto kern = bsa_kernel<D, BN, FP8, PAGED, DENSE, PART, SHKV, LSEX>;
-  cudaError_t e = set_smem_once<bsa_kernel<D, BN, FP8, PAGED, DENSE, PART, SHKV, LSEX>>(C::SMEM_LAUNCH);
+  auto kern = bsa_kernel<D, BN, FP8, PAGED, DENSE, PART, SHKV, LSEX, SNAKE>;
+  cudaError_t e = set_smem_once<bsa_kernel<D, BN, FP8, PAGED, DENSE, PART, SHKV, LSEX, SNAKE>>(C::SMEM_LAUNCH);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
@@ -737,12 +751,12 @@ cudaError_t run_k(const BsaParams& prm, cudaStream_t st) {
 
 // The FP8 first-row launch with a log-sum-exp requested keeps the unrounded P sums beside
 // the rounded ones it normalises by (its own kernel, so the default one carries none of it)
-template <int D, int BN, bool FP8, bool PAGED, bool DENSE, int PART, bool SHKV = false>
+template <int D, int BN, bool FP8, bool PAGED, bool DENSE, int PART, bool SHKV = false, bool SNAKE = false>
 cudaError_t run(const BsaParams& prm, cudaStream_t st) {
   if constexpr (FP8 && PART == kFirstRow) {
-    if (prm.lse != nullptr) return run_k<D, BN, FP8, PAGED, DENSE, PART, SHKV, true>(prm, st);
+    if (prm.lse != nullptr) return run_k<D, BN, FP8, PAGED, DENSE, PART, SHKV, true, SNAKE>(prm, st);
   }
-  return run_k<D, BN, FP8, PAGED, DENSE, PART, SHKV, false>(prm, st);
+  return run_k<D, BN, FP8, PAGED, DENSE, PART, SHKV, false, SNAKE>(prm, st);
 }
 
 template <int D, int BN, bool FP8, int PART>
@@ -755,6 +769,11 @@ cudaError_t run_part(const BsaParams& prm, bool paged, bool dense, cudaStream_t 
   }
   if (paged)
     return dense ? run<D, BN, FP8, true, true, PART>(prm, st) : run<D, BN, FP8, true, false, PART>(prm, st);
+  // an odd number of groups (e.g. a single head pair): the snake order (snake_unit); kept
+  // out of the other kernels, whose round-robin loop it would otherwise slow
+  if constexpr (PART != kFirstRow) {
+    if (!dense && prm.groups % 2 == 1) return run<D, BN, FP8, false, false, PART, false, true>(prm, st);
+  }
   return dense ? run<D, BN, FP8, false, true, PART>(prm, st) : run<D, BN, FP8, false, false, PART>(prm, st);
 }
 

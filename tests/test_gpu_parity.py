@@ -44,6 +44,11 @@ SMALL = {
         110, 275, 73, 15, 223, 27, 163, 228, 51, 138, 173, 233, 150, 162, 166, 139, 10, 286, 250,
         111, 110, 194, 267, 163, 82, 34),
                                     num_q_heads=4, num_kv_heads=2, seed=20),
+    # an odd number of (sequence, head pair) groups, with more units than SMs: the launches
+    # that deal the units forwards and back
+    "snake_bf16": W.QWEN_32K.with_(name="snake_bf16", seqlens=(9000, 6000, 4000), num_q_heads=2, num_kv_heads=1,
+                                   block=64, seed=21),
+    "snake_fp8": W.LONG_128K_FP8.with_(name="snake_fp8", seqlens=(20000,), num_q_heads=2, num_kv_heads=1, seed=22),
 }
 
 _cache = {}
