@@ -2,7 +2,7 @@
 sanitizer): each output, selection, score and workspace buffer is carved out of a larger
 allocation whose 4 KiB before and after hold a sentinel pattern; after each entry point
 runs, the sentinels must be intact and the read-only inputs unchanged.  The workloads
-cover ragged tails, varlen batches, paging, FP8, d = 64 and block 64."""
+cover ragged tails, varlen batches, paging, FP8, d = 64, block 64 and a single head pair."""
 import pytest
 import torch
 
@@ -24,6 +24,10 @@ CASES = {
                                         seed=73),
     "d64_b64_shared": W.QWEN_32K.with_(name="d64_b64_shared", seqlens=(1000, 64, 1), num_q_heads=4,
                                        num_kv_heads=2, head_dim=64, block=64, shared_lists=True, seed=74),
+    # one head pair, more q-block rows than SMs: the attention launch deals its units
+    # forwards and back (an odd number of groups)
+    "single_pair": W.QWEN_32K.with_(name="single_pair", seqlens=(12000,), num_q_heads=2, num_kv_heads=1,
+                                    block=64, seed=75),
 }
 
 
