@@ -284,7 +284,7 @@ __global__ void __launch_bounds__(kFusedThreads) select_fused_kernel(
   const float* lb = lbar + static_cast<long long>(kh) * R + s.row0;
   for (int j0 = 1; j0 < i; j0 += kFusedChunk) {
     const int nj = min(kFusedChunk, i - j0);
-    __syncthreads();  // the previous round's K̄ rows are no longer read
+    __syncthreads();  // the previous chunk's K̄ rows are no longer read
     for (int e = threadIdx.x; e < nj * (D / 4); e += kFusedThreads) {
       const int r = e / (D / 4), c = e % (D / 4);
       *reinterpret_cast<float4*>(Ks + r * L::KS + 4 * c) =
