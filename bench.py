@@ -529,7 +529,10 @@ def sweep(wl, steps, warmup):
 
 
 def run_sweep_only(args):
-    wl = W.ALL[args.workload] if args.workload != W.LONG_128K_FP8.name else W.SWEEP_64K
+    if args.sweep_workload is not None:
+        wl = W.ALL[args.sweep_workload]
+    else:
+        wl = W.ALL[args.workload] if args.workload != W.LONG_128K_FP8.name else W.SWEEP_64K
     _, sw = sweep(wl, args.steps, args.warmup)
     sw["metric"] = "BSA latency vs density (linear fit of ms on selected TFLOP)"
     print(json.dumps(sw), flush=True)
@@ -576,6 +579,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads of the suite")
+    ap.add_argument("--sweep-workload", default=None, choices=sorted(W.ALL),
+                    help="the workload --sweep runs on (default: the 64K BF16 layer)")
     ap.add_argument("--sweep", action="store_true", help="only the density sweep (keep 1.0 .. 0.1) against the dense kernel")
     args = ap.parse_args()
     if args.warmup < 3:
